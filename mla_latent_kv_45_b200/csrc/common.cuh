@@ -1,0 +1,78 @@
+// Shared device helpers for the MLA decode kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mla {
+
+// Bits of the workspace error word.
+enum : int { kErrRange = 1, kErrTimeout = 2 };
+
+// RoPE frequencies theta_i = base^(-2i/d_rope), computed on the host in fp64
+// ("解耦 RoPE（MLA 下）" §七 rope; "从零理解 MLA", 解耦 RoPE precompute_cos_sin).
+// The angle pos * theta_i is formed and its cos / sin evaluated in fp64 on the
+// device, then rounded to fp32, so large positions keep full angle accuracy.
+struct RopeParams {
+  double theta[64];
+  int d_rope;
+  int half;  // 0: pairs (2i, 2i+1); 1: pairs (i, i + d_rope/2)
+};
+
+__device__ __forceinline__ float ld_f(const float *p) { return *p; }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+template <class T> __device__ __forceinline__ T st_cast(float v);
+template <> __device__ __forceinline__ float st_cast<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 st_cast<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ void set_error(int *err, int bit) { atomicOr(err, bit); }
+
+// Rotates the pair (x0, x1) by pos * theta_i.
+__device__ __forceinline__ void rope_pair(const RopeParams &rp, int i, int pos, float &x0,
+                                          float &x1) {
+  double s, c;
+  sincos((double)pos * rp.theta[i], &s, &c);
+  const float cf = (float)c, sf = (float)s;
+  const float a = x0, b = x1;
+  x0 = a * cf - b * sf;
+  x1 = a * sf + b * cf;
+}
+
+// Indices of the two members of RoPE pair i for width d.
+__device__ __forceinline__ void rope_idx(const RopeParams &rp, int i, int &j0, int &j1) {
+  if (rp.half) {
+    j0 = i;
+    j1 = i + rp.d_rope / 2;
+  } else {
+    j0 = 2 * i;
+    j1 = 2 * i + 1;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Per-call plan of the balanced split of a batch's cache pages into partitions.
+// Written by the plan kernel into the workspace, read by the attention and
+// combine kernels.
+struct PlanHeader {
+  int total_pages;   // sum over sequences of ceil(len / page_size)
+  int quota;         // pages per partition (last one may hold fewer)
+  int parts;         // partitions with work
+  int num_partials;  // partial slots used by split sequences
+};
+
+}  // namespace mla

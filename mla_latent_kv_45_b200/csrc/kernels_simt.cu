@@ -1,0 +1,484 @@
+// Generic CUDA-core kernels of the MLA decode step.
+//
+// These kernels accept any small head / latent sizes.  In fp32 they are the
+// validation path (every step computed in fp32, one rounding per stored
+// value).  The plan and combine kernels are shared with the sm_100a
+// tensor-core attention kernel.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// Skinny matrix products  Y[b][m] = sum_k W[m][k] X[b][k]   (per head z)
+// ---------------------------------------------------------------------------
+
+// W contiguous along k: one warp per output row m, lanes stride over k, eight
+// batch rows at a time.
+template <class TW, class TX, class TY>
+__global__ void gemv_k_contig(GemvArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int head = blockIdx.z;
+  if (m >= a.M) return;
+  const TW *w = reinterpret_cast<const TW *>(a.W) + head * a.w_head + (long)m * a.w_m;
+  const TX *x = reinterpret_cast<const TX *>(a.X) + head * a.x_head;
+  TY *y = reinterpret_cast<TY *>(a.Y) + head * a.y_head;
+  for (int b0 = blockIdx.y * 8; b0 < a.B; b0 += gridDim.y * 8) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    for (int k = lane; k < a.K; k += 32) {
+      const float wv = ld_f(w + k);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (b0 + j < a.B) acc[j] += wv * ld_f(x + (long)(b0 + j) * a.x_b + k);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float v = warp_sum(acc[j]);
+      if (lane == 0 && b0 + j < a.B) y[(long)(b0 + j) * a.y_b + m] = st_cast<TY>(v);
+    }
+  }
+}
+
+// W contiguous along m (a transposed weight, e.g. W_UK,i^T): one thread per
+// output m, the batch rows' x staged in shared memory.
+template <class TW, class TX, class TY>
+__global__ void gemv_m_contig(GemvArgs a) {
+  extern __shared__ float xs[];  // [8][K]
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  const int head = blockIdx.z;
+  const TW *w = reinterpret_cast<const TW *>(a.W) + head * a.w_head;
+  const TX *x = reinterpret_cast<const TX *>(a.X) + head * a.x_head;
+  TY *y = reinterpret_cast<TY *>(a.Y) + head * a.y_head;
+  for (int b0 = blockIdx.y * 8; b0 < a.B; b0 += gridDim.y * 8) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < 8 * a.K; i += blockDim.x) {
+      const int j = i / a.K, k = i % a.K;
+      xs[i] = (b0 + j < a.B) ? ld_f(x + (long)(b0 + j) * a.x_b + k) : 0.f;
+    }
+    __syncthreads();
+    if (m < a.M) {
+      float acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+      for (int k = 0; k < a.K; ++k) {
+        const float wv = ld_f(w + (long)k * a.w_k + m);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += wv * xs[j * a.K + k];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (b0 + j < a.B) y[(long)(b0 + j) * a.y_b + m] = st_cast<TY>(acc[j]);
+    }
+  }
+}
+
+template <class TW, class TX, class TY>
+cudaError_t launch_gemv(const GemvArgs &a, int heads, cudaStream_t s) {
+  const int bgrid = (a.B + 7) / 8 < 64 ? (a.B + 7) / 8 : 64;
+  if (a.w_k == 1) {
+    dim3 grid((a.M + 7) / 8, bgrid, heads);
+    gemv_k_contig<TW, TX, TY><<<grid, 256, 0, s>>>(a);
+  } else {
+    dim3 grid((a.M + 127) / 128, bgrid, heads);
+    gemv_m_contig<TW, TX, TY><<<grid, 128, 8 * a.K * sizeof(float), s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+#define MLA_INST_GEMV(TW, TX, TY) \
+  template cudaError_t launch_gemv<TW, TX, TY>(const GemvArgs &, int, cudaStream_t);
+MLA_INST_GEMV(float, float, float)
+MLA_INST_GEMV(__nv_bfloat16, __nv_bfloat16, float)
+MLA_INST_GEMV(__nv_bfloat16, float, float)
+MLA_INST_GEMV(__nv_bfloat16, float, __nv_bfloat16)
+MLA_INST_GEMV(__nv_bfloat16, __nv_bfloat16, __nv_bfloat16)
+
+// ---------------------------------------------------------------------------
+// Cache-append epilogue: RMSNorm on c, RoPE on k_R, one rounding, paged write
+// ---------------------------------------------------------------------------
+
+template <class T>
+__global__ void append_finish(const float *xkv, int d_c, RopeParams rp, const T *gamma,
+                              float eps, const int32_t *positions, T *pool, int num_pages,
+                              int page_size, const int32_t *block_table, int max_pages,
+                              int *err) {
+  const int b = blockIdx.x;
+  const int row = d_c + rp.d_rope;
+  const float *x = xkv + (long)b * row;
+  __shared__ float red[32];
+  __shared__ float inv_rms;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss += x[i] * x[i];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) inv_rms = 1.0f / sqrtf(v / (float)d_c + eps);
+  }
+  __syncthreads();
+  const int pos = positions[b];
+  const long cap = (long)max_pages * page_size;
+  int page = -1;
+  if (pos >= 0 && pos < cap) page = block_table[(long)b * max_pages + pos / page_size];
+  if (page < 0 || page >= num_pages) {
+    if (threadIdx.x == 0) set_error(err, kErrRange);
+    return;
+  }
+  T *dst = pool + ((long)page * page_size + pos % page_size) * row;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x)
+    dst[i] = st_cast<T>(ld_f(gamma + i) * (x[i] * inv_rms));
+  for (int i = threadIdx.x; i < rp.d_rope / 2; i += blockDim.x) {
+    int j0, j1;
+    rope_idx(rp, i, j0, j1);
+    float x0 = x[d_c + j0], x1 = x[d_c + j1];
+    rope_pair(rp, i, pos, x0, x1);
+    dst[d_c + j0] = st_cast<T>(x0);
+    dst[d_c + j1] = st_cast<T>(x1);
+  }
+}
+
+template <class T>
+cudaError_t launch_append_finish(const float *xkv, int batch, int d_c, const RopeParams &rp,
+                                 const T *gamma, float eps, const int32_t *positions, T *pool,
+                                 int num_pages, int page_size, const int32_t *block_table,
+                                 int max_pages, int *err, cudaStream_t s) {
+  append_finish<T><<<batch, 256, 0, s>>>(xkv, d_c, rp, gamma, eps, positions, pool, num_pages,
+                                          page_size, block_table, max_pages, err);
+  return cudaGetLastError();
+}
+template cudaError_t launch_append_finish<float>(const float *, int, int, const RopeParams &,
+                                                 const float *, float, const int32_t *, float *,
+                                                 int, int, const int32_t *, int, int *,
+                                                 cudaStream_t);
+template cudaError_t launch_append_finish<__nv_bfloat16>(
+    const float *, int, int, const RopeParams &, const __nv_bfloat16 *, float, const int32_t *,
+    __nv_bfloat16 *, int, int, const int32_t *, int, int *, cudaStream_t);
+
+// ---------------------------------------------------------------------------
+// q_R = RoPE_pos(W_QR c_Q) written into the tail of each q_lat row
+// ---------------------------------------------------------------------------
+
+template <class T>
+__global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
+                       const int32_t *positions, T *q_lat) {
+  const int b = blockIdx.x;
+  const int half = rp.d_rope / 2;
+  const int pos = positions[b];
+  for (int t = threadIdx.x; t < n_heads * half; t += blockDim.x) {
+    const int h = t / half, i = t % half;
+    int j0, j1;
+    rope_idx(rp, i, j0, j1);
+    const float *src = qr + ((long)b * n_heads + h) * rp.d_rope;
+    float x0 = src[j0], x1 = src[j1];
+    rope_pair(rp, i, pos, x0, x1);
+    T *dst = q_lat + ((long)b * n_heads + h) * (d_c + rp.d_rope) + d_c;
+    dst[j0] = st_cast<T>(x0);
+    dst[j1] = st_cast<T>(x1);
+  }
+}
+
+template <class T>
+cudaError_t launch_rope_q(const float *qr, int batch, int n_heads, int d_c, const RopeParams &rp,
+                          const int32_t *positions, T *q_lat, cudaStream_t s) {
+  rope_q<T><<<batch, 256, 0, s>>>(qr, n_heads, d_c, rp, positions, q_lat);
+  return cudaGetLastError();
+}
+template cudaError_t launch_rope_q<float>(const float *, int, int, int, const RopeParams &,
+                                          const int32_t *, float *, cudaStream_t);
+template cudaError_t launch_rope_q<__nv_bfloat16>(const float *, int, int, int,
+                                                  const RopeParams &, const int32_t *,
+                                                  __nv_bfloat16 *, cudaStream_t);
+
+// ---------------------------------------------------------------------------
+// Plan: balanced split of the batch's pages into partitions
+// ---------------------------------------------------------------------------
+//
+// Sequence b holds n_b = ceil(len_b / page_size) pages.  Concatenating all
+// sequences' pages gives N pages; partition p takes global pages
+// [p*quota, (p+1)*quota).  A sequence cut by a partition boundary is computed
+// in pieces whose unnormalised partials are merged by the combine kernel.
+
+__global__ void plan_kernel(PlanArgs a) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x;
+  const long cap = (long)a.max_pages * a.page_size;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  // pass 1: page counts, validity, exclusive prefix sum -> seq_start
+  for (int base = 0; base < a.batch; base += blockDim.x) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < a.batch) {
+      const int len = a.seq_lens[b];
+      const bool ok = len > 0 && len <= cap;
+      n = ok ? (len + a.page_size - 1) / a.page_size : 0;
+      a.bad[b] = ok ? 0 : 1;
+      if (!ok) set_error(a.err, kErrRange);
+    }
+    // block-wide inclusive scan of n
+    int v = n;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if ((tid & 31) >= o) v += t;
+    }
+    if ((tid & 31) == 31) warp_tot[tid >> 5] = v;
+    __syncthreads();
+    if (tid < 32) {
+      int w = tid < (blockDim.x >> 5) ? warp_tot[tid] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, w, o);
+        if (tid >= o) w += t;
+      }
+      warp_tot[tid] = w;
+    }
+    __syncthreads();
+    const int incl = v + ((tid >> 5) ? warp_tot[(tid >> 5) - 1] : 0) + carry;
+    if (b < a.batch) a.seq_start[b] = incl - n;
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  __shared__ int quota;
+  if (tid == 0) {
+    const int N = carry;
+    a.seq_start[a.batch] = N;
+    int parts = 0, q = 1;
+    if (N > 0) {
+      int p = a.parts_max;
+      const int by_min = (N + a.min_pages - 1) / a.min_pages;
+      if (p > by_min) p = by_min;
+      if (p < 1) p = 1;
+      q = (N + p - 1) / p;
+      parts = (N + q - 1) / q;
+    }
+    a.hdr->total_pages = N;
+    a.hdr->quota = q;
+    a.hdr->parts = parts;
+    quota = q;
+    carry = 0;
+  }
+  __syncthreads();
+  // pass 2: pieces per sequence and partial-slot bases
+  for (int base = 0; base < a.batch; base += blockDim.x) {
+    const int b = base + tid;
+    int pieces = 0;
+    if (b < a.batch) {
+      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+      if (s1 > s0) pieces = (s1 - 1) / quota - s0 / quota + 1;
+    }
+    const int n = pieces > 1 ? pieces : 0;
+    int v = n;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if ((tid & 31) >= o) v += t;
+    }
+    if ((tid & 31) == 31) warp_tot[tid >> 5] = v;
+    __syncthreads();
+    if (tid < 32) {
+      int w = tid < (blockDim.x >> 5) ? warp_tot[tid] : 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, w, o);
+        if (tid >= o) w += t;
+      }
+      warp_tot[tid] = w;
+    }
+    __syncthreads();
+    const int incl = v + ((tid >> 5) ? warp_tot[(tid >> 5) - 1] : 0) + carry;
+    if (b < a.batch) a.part_base[b] = n ? incl - n : -1;
+    __syncthreads();
+    if (tid == blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  if (tid == 0) a.hdr->num_partials = carry;
+}
+
+cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s) {
+  plan_kernel<<<1, 1024, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core latent attention (any small sizes): one block per (partition, head)
+// ---------------------------------------------------------------------------
+
+template <class T>
+__global__ void attn_simt(AttnArgs a) {
+  constexpr int NT = 128;
+  const int p = blockIdx.x, h = blockIdx.y;
+  const PlanHeader hdr = *a.hdr;
+  if (p >= hdr.parts) return;
+  const int row = a.d_c + a.d_rope;
+  extern __shared__ float sm[];
+  float *qs = sm;              // [row]
+  float *ps = qs + row;        // [NT]
+  int *pg = reinterpret_cast<int *>(ps + NT);  // [NT]
+  __shared__ float red[NT / 32];
+  const T *pool = reinterpret_cast<const T *>(a.pool);
+  constexpr int MAXD = 8;  // d_c <= MAXD * NT
+  const int g1 = min(hdr.total_pages, (p + 1) * hdr.quota);
+  int g0 = p * hdr.quota;
+  // first sequence: largest b with seq_start[b] <= g0
+  int lo = 0, hi = a.batch;  // invariant seq_start[lo] <= g0 < seq_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.seq_start[mid] <= g0) lo = mid; else hi = mid;
+  }
+  int b = lo;
+  while (g0 < g1) {
+    const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+    if (s1 <= g0) { ++b; continue; }
+    const int lp1 = min(g1, s1) - s0;
+    const int len = a.seq_lens[b];
+    const int r_begin = (g0 - s0) * a.page_size;
+    const int r_end = min(lp1 * a.page_size, len);
+    const T *q = reinterpret_cast<const T *>(a.q_lat) + ((long)b * a.n_heads + h) * row;
+    __syncthreads();
+    for (int j = threadIdx.x; j < row; j += NT) qs[j] = ld_f(q + j);
+    __syncthreads();
+    float m = -INFINITY, l = 0.f, acc[MAXD];
+#pragma unroll
+    for (int k = 0; k < MAXD; ++k) acc[k] = 0.f;
+    for (int r0 = r_begin; r0 < r_end; r0 += NT) {
+      const int s = r0 + threadIdx.x;
+      float logit = -INFINITY;
+      if (s < r_end) {
+        int page = a.block_table[(long)b * a.max_pages + s / a.page_size];
+        if (page < 0 || page >= a.num_pages) {
+          set_error(a.err, kErrRange);
+          a.bad[b] = 1;
+          page = 0;
+        }
+        pg[threadIdx.x] = page;
+        const T *rp = pool + ((long)page * a.page_size + s % a.page_size) * row;
+        float dot = 0.f;
+        for (int j = 0; j < row; ++j) dot += qs[j] * ld_f(rp + j);
+        logit = dot * a.scale;
+      }
+      float cm = warp_max(logit);
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cm;
+      __syncthreads();
+      cm = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      __syncthreads();
+      const float m_new = fmaxf(m, cm);
+      const float alpha = expf(m - m_new);
+      const float pv = (s < r_end) ? expf(logit - m_new) : 0.f;
+      ps[threadIdx.x] = pv;
+      float cs = warp_sum(pv);
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cs;
+      __syncthreads();
+      cs = red[0] + red[1] + red[2] + red[3];
+      l = l * alpha + cs;
+      m = m_new;
+      const int n = min(NT, r_end - r0);
+#pragma unroll
+      for (int k = 0; k < MAXD; ++k) {
+        const int d = threadIdx.x + k * NT;
+        if (d < a.d_c) {
+          float v = acc[k] * alpha;
+          for (int t = 0; t < n; ++t) {
+            const int st = r0 + t;
+            v += ps[t] * ld_f(pool + ((long)pg[t] * a.page_size + st % a.page_size) * row + d);
+          }
+          acc[k] = v;
+        }
+      }
+      __syncthreads();
+    }
+    const int pb = a.part_base[b];
+    if (pb < 0) {
+      T *z = reinterpret_cast<T *>(a.z) + ((long)b * a.n_heads + h) * a.d_c;
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int k = 0; k < MAXD; ++k) {
+        const int d = threadIdx.x + k * NT;
+        if (d < a.d_c) z[d] = st_cast<T>(acc[k] * inv);
+      }
+      if (a.lse && threadIdx.x == 0) a.lse[(long)b * a.n_heads + h] = m + logf(l);
+    } else {
+      const int slot = pb + (p - s0 / hdr.quota);
+      float *O = a.part_O + ((long)slot * a.n_heads + h) * a.d_c;
+#pragma unroll
+      for (int k = 0; k < MAXD; ++k) {
+        const int d = threadIdx.x + k * NT;
+        if (d < a.d_c) O[d] = acc[k];
+      }
+      if (threadIdx.x == 0) {
+        a.part_m[(long)slot * a.n_heads + h] = m;
+        a.part_l[(long)slot * a.n_heads + h] = l;
+      }
+    }
+    g0 = s0 + lp1;
+    ++b;
+  }
+}
+
+template <class T>
+cudaError_t launch_attn_simt(const AttnArgs &a, int parts_max, cudaStream_t s) {
+  const size_t smem = (a.d_c + a.d_rope + 128) * sizeof(float) + 128 * sizeof(int);
+  dim3 grid(parts_max, a.n_heads);
+  attn_simt<T><<<grid, 128, smem, s>>>(a);
+  return cudaGetLastError();
+}
+template cudaError_t launch_attn_simt<float>(const AttnArgs &, int, cudaStream_t);
+template cudaError_t launch_attn_simt<__nv_bfloat16>(const AttnArgs &, int, cudaStream_t);
+
+// ---------------------------------------------------------------------------
+// Combine split partials; zero the outputs of invalid sequences
+// ---------------------------------------------------------------------------
+//
+// z = sum_j w_j O_j / sum_j w_j l_j with w_j = exp(m_j - max_j m_j), and
+// lse = max_j m_j + log(sum_j w_j l_j): the standard merge of partial softmaxes.
+
+template <class T>
+__global__ void combine_kernel(AttnArgs a) {
+  const int b = blockIdx.x;
+  const PlanHeader hdr = *a.hdr;
+  T *zb = reinterpret_cast<T *>(a.z) + (long)b * a.n_heads * a.d_c;
+  if (a.bad[b]) {
+    for (int i = threadIdx.x; i < a.n_heads * a.d_c; i += blockDim.x) zb[i] = st_cast<T>(0.f);
+    if (a.lse)
+      for (int h = threadIdx.x; h < a.n_heads; h += blockDim.x)
+        a.lse[(long)b * a.n_heads + h] = -INFINITY;
+    return;
+  }
+  const int pb = a.part_base[b];
+  if (pb < 0) return;
+  const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+  const int pieces = (s1 - 1) / hdr.quota - s0 / hdr.quota + 1;
+  for (int h = blockIdx.y; h < a.n_heads; h += gridDim.y) {
+    float M = -INFINITY;
+    for (int j = 0; j < pieces; ++j) M = fmaxf(M, a.part_m[(long)(pb + j) * a.n_heads + h]);
+    float den = 0.f;
+    for (int j = 0; j < pieces; ++j) {
+      const long idx = (long)(pb + j) * a.n_heads + h;
+      den += expf(a.part_m[idx] - M) * a.part_l[idx];
+    }
+    const float inv = 1.f / den;
+    for (int d = threadIdx.x; d < a.d_c; d += blockDim.x) {
+      float v = 0.f;
+      for (int j = 0; j < pieces; ++j) {
+        const long idx = (long)(pb + j) * a.n_heads + h;
+        v += expf(a.part_m[idx] - M) * a.part_O[idx * a.d_c + d];
+      }
+      zb[(long)h * a.d_c + d] = st_cast<T>(v * inv);
+    }
+    if (a.lse && threadIdx.x == 0) a.lse[(long)b * a.n_heads + h] = M + logf(den);
+  }
+}
+
+template <class T>
+cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s) {
+  dim3 grid(a.batch, a.n_heads < 16 ? a.n_heads : 16);
+  combine_kernel<T><<<grid, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+template cudaError_t launch_combine<float>(const AttnArgs &, cudaStream_t);
+template cudaError_t launch_combine<__nv_bfloat16>(const AttnArgs &, cudaStream_t);
+
+}  // namespace mla

@@ -1,0 +1,54 @@
+"""One decode step of an MLA layer through the four C-ABI calls.
+
+The order is the pages' per-token inference flow ("解耦 RoPE（MLA 下）" §五):
+append the new token's [c ; k_R] row, build the absorbed query, attend over
+the whole cache (the new row included), then up-project.  Device tensors only;
+every step runs in the CUDA library.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib as L
+
+
+class DecodeLayer:
+    """Weights of one layer (device tensors, ``[out, in]`` layout) plus a workspace."""
+
+    def __init__(self, dims: L.Dims, weights: dict, batch: int, num_splits: int = 0,
+                 device="cuda"):
+        self.dims = dims
+        self.w = weights
+        self.batch = batch
+        self.num_splits = num_splits
+        self.d_model = weights["W_DKV"].shape[1]
+        self.d_q = weights["W_DQ"].shape[0] if weights.get("W_DQ") is not None else 0
+        nbytes = L.mla_workspace_size(dims, batch, self.d_model, self.d_q, num_splits)
+        if nbytes == 0:
+            raise ValueError("unsupported dims for the workspace")
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        L.mla_workspace_init(self.ws)
+        H, dt = dims.n_heads, dims.torch_dtype
+        self.q_lat = torch.empty(batch, H, dims.d_c + dims.d_rope, dtype=dt, device=device)
+        self.z = torch.empty(batch, H, dims.d_c, dtype=dt, device=device)
+        self.lse = torch.empty(batch, H, dtype=torch.float32, device=device)
+        d_out = self.d_model if weights.get("W_O") is not None else H * dims.d_v
+        self.out = torch.empty(batch, d_out, dtype=dt, device=device)
+
+    def step(self, cache: L.PagedCache, h: torch.Tensor, positions: torch.Tensor,
+             stream=None) -> torch.Tensor:
+        """Appends h's rows at ``positions`` and returns the layer output.
+
+        ``cache.seq_lens`` must already count the new rows (positions + 1).
+        """
+        w, d = self.w, self.dims
+        L.mla_cache_append(d, cache, h, w["W_DKV"], w["W_KR"], w["gamma"], positions, self.ws,
+                           stream)
+        L.mla_absorb_q(d, h, w.get("W_DQ"), w["W_UQ"], w["W_QR"], w["W_UK"], positions,
+                       self.q_lat, self.ws, stream)
+        L.mla_decode_attn(d, cache, self.q_lat, self.z, self.lse, self.num_splits, self.ws, stream)
+        L.mla_unabsorb_out(d, self.z, w["W_UV"], w.get("W_O"), self.out, self.ws, stream)
+        return self.out
