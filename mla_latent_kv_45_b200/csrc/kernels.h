@@ -73,3 +73,48 @@ template <class T>
 cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s);
 
 }  // namespace mla
+
+namespace mla {
+
+// One piece of a partition: local pages [lp0, lp1) of sequence b (s0 = the
+// sequence's first global page, len = its row count).
+struct Segment {
+  int b, lp0, lp1, len, s0;
+};
+
+// Walks the segments of partition p of the plan (global pages
+// [p*quota, (p+1)*quota) of the batch's concatenated page list).
+struct SegmentWalker {
+  int g0, g1, b;
+
+  __device__ __forceinline__ void init(const AttnArgs &a, const PlanHeader &h, int p) {
+    g0 = p * h.quota;
+    g1 = min(h.total_pages, g0 + h.quota);
+    b = 0;
+    if (g0 >= g1) return;
+    int lo = 0, hi = a.batch;  // seq_start[lo] <= g0 < seq_start[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.seq_start[mid] <= g0) lo = mid; else hi = mid;
+    }
+    b = lo;
+  }
+
+  __device__ __forceinline__ bool next(const AttnArgs &a, Segment &s) {
+    while (g0 < g1) {
+      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+      if (s1 <= g0) { ++b; continue; }
+      s.b = b;
+      s.s0 = s0;
+      s.lp0 = g0 - s0;
+      s.lp1 = min(g1, s1) - s0;
+      s.len = a.seq_lens[b];
+      g0 = s0 + s.lp1;
+      ++b;
+      return true;
+    }
+    return false;
+  }
+};
+
+}  // namespace mla

@@ -426,7 +426,6 @@ cudaError_t launch_attn_simt(const AttnArgs &a, int parts_max, cudaStream_t s) {
   return cudaGetLastError();
 }
 template cudaError_t launch_attn_simt<float>(const AttnArgs &, int, cudaStream_t);
-template cudaError_t launch_attn_simt<__nv_bfloat16>(const AttnArgs &, int, cudaStream_t);
 
 // ---------------------------------------------------------------------------
 // Combine split partials; zero the outputs of invalid sequences
