@@ -169,6 +169,29 @@ mla_status mla_unabsorb_out(const mla_dims *dims, int batch, const void *z, cons
                             const void *W_O, int d_model, void *out, void *ws, size_t ws_bytes,
                             mla_stream_t stream);
 
+/* Decode attention without a caller-provided workspace.  The pages describe no
+ * such variant: it exists for callers that cannot allocate device memory, e.g.
+ * code whose device memory belongs entirely to another allocator (a
+ * framework's caching pool or an arena reserved at start-up) or a plugin
+ * interface that hands over only the operation's tensors and allows no
+ * allocation while it runs.
+ * Computes exactly what mla_decode_attn computes, with the same arguments
+ * minus the workspace.  Its scratch (plan, split-KV partials, error word) is a
+ * fixed 16 MiB array inside the library, present on every device that loads
+ * the library until the process exits.  num_splits = 0 picks the most
+ * partitions that fit (at most one per pair of SMs); a batch or num_splits
+ * whose scratch would exceed 16 MiB returns MLA_ERR_WORKSPACE before any work
+ * is enqueued (for the bf16 sizes: about 60 partitions at small batch).
+ * The first call on a device looks up the array's device address for that
+ * device; make it before any stream capture.  Calls share the array: calls
+ * whose work overlaps on the GPU race and must be serialised by the caller.
+ * Device-side range errors zero the affected sequence (z = 0, lse = -inf) as in
+ * mla_decode_attn; the error word itself is cleared at the start of each call
+ * and is not readable by the caller. */
+mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_paged_cache *cache, int batch,
+                                   const void *q_lat, void *z, float *lse, int num_splits,
+                                   mla_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns MLA_OK, MLA_ERR_DEVICE_RANGE or MLA_ERR_TIMEOUT (or MLA_ERR_CUDA if
  * the stream itself failed).  This is the only call that synchronises. */

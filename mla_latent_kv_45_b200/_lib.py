@@ -26,7 +26,8 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
           6: "MLA_ERR_DEVICE_RANGE", 7: "MLA_ERR_TIMEOUT"}
 
 EXPORTS = ("mla_workspace_size", "mla_workspace_init", "mla_cache_append", "mla_absorb_q",
-           "mla_decode_attn", "mla_unabsorb_out", "mla_get_device_error", "mla_status_string")
+           "mla_decode_attn", "mla_decode_attn_noalloc", "mla_unabsorb_out",
+           "mla_get_device_error", "mla_status_string")
 
 
 class MlaError(RuntimeError):
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
         L.mla_cache_append.argtypes = [pd, pc, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.mla_absorb_q.argtypes = [pd, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.mla_decode_attn.argtypes = [pd, pc, i, vp, vp, vp, i, vp, sz, vp]
+        L.mla_decode_attn_noalloc.argtypes = [pd, pc, i, vp, vp, vp, i, vp]
         L.mla_unabsorb_out.argtypes = [pd, i, vp, vp, vp, i, vp, vp, sz, vp]
         L.mla_get_device_error.argtypes = [vp, vp]
         L.mla_status_string.argtypes = [i]
@@ -170,6 +172,15 @@ def mla_decode_attn(dims: Dims, cache: PagedCache, q_lat, z, lse=None, num_split
     _ok("mla_decode_attn", lib().mla_decode_attn(
         ctypes.byref(d), ctypes.byref(c), q_lat.shape[0], _p(q_lat), _p(z), _p(lse), num_splits,
         _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def mla_decode_attn_noalloc(dims: Dims, cache: PagedCache, q_lat, z, lse=None,
+                            num_splits: int = 0, stream=None):
+    """Decode attention with the library's fixed internal scratch (no workspace)."""
+    d, c = dims.c(), cache.c()
+    _ok("mla_decode_attn_noalloc", lib().mla_decode_attn_noalloc(
+        ctypes.byref(d), ctypes.byref(c), q_lat.shape[0], _p(q_lat), _p(z), _p(lse), num_splits,
+        _stream(stream)))
 
 
 def mla_unabsorb_out(dims: Dims, z, W_UV, W_O, out, ws: torch.Tensor, stream=None):
