@@ -1,0 +1,346 @@
+// Skinny bf16 GEMMs of the decode projections on sm_100a tensor cores.
+//
+// Y[n][m] = sum_k A[m][k] X[n][k] with m over the weight's output rows, n over
+// the batch (N <= 256) and k over the input width.  Decode projections are
+// weight-bandwidth bound (each weight element is used B times), so the design
+// streams the weights once through a deep TMA ring with as many CTAs as it
+// takes to keep HBM busy:
+//  * each CTA owns one 128-row tile of one problem and a K range (split-K);
+//    D = A_tile . X^T accumulates in TMEM (tcgen05.mma, M = 128, N = batch
+//    padded to 16, K = 16 per instruction);
+//  * A comes K-major ([out][in] weights) or MN-major (a per-head transposed
+//    view such as W_UK,i^T) -- both through 128-byte-swizzled TMA boxes;
+//  * X (the activations, bf16) is reloaded from L2 per K chunk;
+//  * several problems that share X (e.g. W_DKV and W_KR, W_UQ and W_QR) run
+//    in one launch; per-head problems (W_UK, W_UV) index heads in the grid;
+//  * the epilogue writes bf16 / fp32 outputs directly or fp32 split-K
+//    partials that gemm_reduce sums in a fixed order (deterministic).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue,
+// warps 2-5 epilogue.  Every wait is bounded (globaltimer).
+#include <cuda.h>
+
+#include "ptx.cuh"
+#include "sm100.h"
+#include "gemm_sm100.h"
+
+namespace mla {
+namespace sm100 {
+namespace {
+
+using namespace ptx;
+
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kABytes = 128 * 128;  // 128 rows x 64 bf16
+
+struct Bars {
+  uint64_t full[kMaxGemmStages], empty[kMaxGemmStages], d_full, drain;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+__device__ __forceinline__ bool gwait(Bars *bars, int *err, uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(a, parity)) return true;
+    if (bars->abort) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      set_error(err, kErrTimeout);
+      bars->abort = 1;
+      return false;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    gemm_sm100_kernel(const __grid_constant__ CUtensorMap tm_a0,
+                      const __grid_constant__ CUtensorMap tm_a1,
+                      const __grid_constant__ CUtensorMap tm_x, const GemmLaunch g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int stage_bytes = kABytes + g.n_pad * 128;
+  Bars *bars = reinterpret_cast<Bars *>(smem + g.stages * stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // which problem / tile / split / head this CTA computes
+  int pi = 0;
+  while (pi + 1 < g.nprob && (int)blockIdx.x >= g.p[pi + 1].tile_begin) ++pi;
+  const GemmProblem &P = g.p[pi];
+  int t = blockIdx.x - P.tile_begin;
+  const int m_tile = t % P.m_tiles;
+  t /= P.m_tiles;
+  const int split = t % P.splits;
+  const int head = t / P.splits;
+  const int m0 = m_tile * 128;
+  const int kc0 = split * P.chunks_per_split;
+  const int kc1 = min(g.k_chunks, kc0 + P.chunks_per_split);
+  const int nk = kc1 - kc0;
+  const CUtensorMap *tm_a = P.a_map ? &tm_a1 : &tm_a0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < g.stages; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->d_full, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(tm_a);
+    prefetch_tmap(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, g.tmem_cols);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int tx = kABytes + g.n_pad * 128;
+      int issued = 0;
+      for (int i = 0; i < nk; ++i, ++issued) {
+        const int st = i % g.stages;
+        if (i >= g.stages && !gwait(bars, g.err, &bars->empty[st], ((i / g.stages) - 1) & 1))
+          break;
+        uint8_t *a_dst = smem + st * stage_bytes;
+        uint8_t *x_dst = a_dst + kABytes;
+        const int k = (kc0 + i) * 64;
+        mbar_expect_tx(&bars->full[st], tx);
+        if (P.a_mn) {
+          // A[m][k] = A2d[head * K + k][m]: two 64-wide MN chunks, 64 K rows each
+          const int y = head * P.a_rows_per_head + k;
+          tma_load_2d(a_dst, tm_a, m0, y, &bars->full[st]);
+          tma_load_2d(a_dst + kABytes / 2, tm_a, m0 + 64, y, &bars->full[st]);
+        } else {
+          tma_load_2d(a_dst, tm_a, k, head * P.a_rows_per_head + m0, &bars->full[st]);
+        }
+        tma_load_2d(x_dst, &tm_x, head * g.x_cols_per_head + k, 0, &bars->full[st]);
+      }
+      for (int i = issued - g.stages; i < issued; ++i)
+        if (i >= 0) gwait(bars, g.err, &bars->full[i % g.stages], (i / g.stages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, g.n_pad, P.a_mn, 0);
+      bool ok = true;
+      for (int i = 0; i < nk; ++i) {
+        const int st = i % g.stages;
+        if (!gwait(bars, g.err, &bars->full[st], (i / g.stages) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + st * stage_bytes);
+        const uint32_t x_base = a_base + kABytes;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = P.a_mn ? sdesc(a_base + 2048 * k, kABytes / 2, 1024, 2)
+                                     : sdesc(a_base + 32 * k, 16, 1024, 2);
+          const uint64_t bd = sdesc(x_base + 32 * k, 16, 1024, 2);
+          umma_bf16(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&bars->empty[st]);
+      }
+      if (ok) umma_commit(&bars->d_full);
+      umma_commit(&bars->drain);
+      gwait(bars, g.err, &bars->drain, 0);
+    }
+  } else {
+    // epilogue: warps 2..5 cover TMEM lanes 64..127, 0..63 (lane quadrant = warp % 4)
+    const int quad = warp & 3;
+    const int ml = quad * 32 + lane;
+    const int m = m0 + ml;
+    if (nk > 0 && gwait(bars, g.err, &bars->d_full, 0)) {
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+      for (int c = 0; c < g.n_pad; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c, r);
+        tmem_wait_ld();
+        if (m < P.M) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = c + j;
+            if (n < g.n) {
+              const float v = __uint_as_float(r[j]);
+              if (P.out_mode == kOutPartial) {
+                P.part[((long)split * g.n_total + g.n0 + n) * P.part_ld + P.part_col +
+                       (long)head * P.M + m] = v;
+              } else {
+                const long idx = (long)n * P.ldy + (long)head * P.y_head + m;
+                if (P.out_mode == kOutBf16)
+                  static_cast<__nv_bfloat16 *>(P.out)[idx] = __float2bfloat16_rn(v);
+                else
+                  static_cast<float *>(P.out)[idx] = v;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, g.tmem_cols);
+  }
+}
+
+// Y[n][col_off + m] = sum over splits of part[s][n][m]  (bf16 or fp32 output)
+__global__ void gemm_reduce_kernel(const float *part, int splits, int n_rows, int width,
+                                   int part_ld, void *out, long ldy, int out_bf16) {
+  const long total = (long)n_rows * width;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
+       i += (long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / width), m = (int)(i % width);
+    float v = 0.f;
+    for (int s = 0; s < splits; ++s) v += part[((long)s * n_rows + n) * part_ld + m];
+    if (out_bf16)
+      static_cast<__nv_bfloat16 *>(out)[(long)n * ldy + m] = __float2bfloat16_rn(v);
+    else
+      static_cast<float *>(out)[(long)n * ldy + m] = v;
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 row-major [rows][cols] map with a box of box_cols x box_rows, 128B swizzle.
+bool map2d(CUtensorMap *m, const void *base, long rows, long cols, int box_cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+int gemm_splits(int m_tiles, int heads, int k_chunks) {
+  // about two resident CTAs per SM, at least 8 K chunks (128 KB of weights) per CTA
+  const int tiles = m_tiles * heads;
+  int s = 2 * sm_count() / tiles;
+  const int max_s = k_chunks / 8 > 0 ? k_chunks / 8 : 1;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  // no empty split: every split gets ceil(k_chunks / s) chunks but the last
+  const int per = (k_chunks + s - 1) / s;
+  return (k_chunks + per - 1) / per;
+}
+
+cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, long x_cols, int K,
+                 int x_cols_per_head, int *err, cudaStream_t s) {
+  if (nops < 1 || nops > 2 || n < 1 || K % 64) return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_sm100_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  for (int n0 = 0; n0 < n; n0 += 256) {
+    const int nn = n - n0 < 256 ? n - n0 : 256;
+    GemmLaunch g{};
+    g.n = nn;
+    g.n0 = n0;
+    g.n_total = n;
+    g.n_pad = (nn + 15) / 16 * 16;
+    g.k_chunks = K / 64;
+    g.x_cols_per_head = x_cols_per_head;
+    g.err = err;
+    g.tmem_cols = 32;
+    while (g.tmem_cols < g.n_pad) g.tmem_cols *= 2;
+    const int stage_bytes = kABytes + g.n_pad * 128;
+    // two CTAs per SM: half of the 227 KB of shared memory each
+    g.stages = (232448 / 2 - 1024 - 256) / stage_bytes;
+    if (g.stages > kMaxGemmStages) g.stages = kMaxGemmStages;
+    CUtensorMap tm[2], tx;
+    int tiles = 0;
+    g.nprob = nops;
+    for (int i = 0; i < nops; ++i) {
+      const GemmOp &o = ops[i];
+      GemmProblem &P = g.p[i];
+      P.M = o.M;
+      P.m_tiles = (o.M + 127) / 128;
+      P.a_mn = o.a_mn;
+      P.a_map = i;
+      P.a_rows_per_head = o.a_mn ? K : o.M;
+      P.splits = o.part ? o.splits : 1;
+      P.chunks_per_split = (g.k_chunks + P.splits - 1) / P.splits;
+      P.tile_begin = tiles;
+      tiles += P.m_tiles * P.splits * o.heads;
+      P.out_mode = o.part ? kOutPartial : o.out_mode;
+      P.out = o.out;
+      P.ldy = o.ldy;
+      P.y_head = o.y_head;
+      P.part = o.part;
+      P.part_ld = o.part_ld;
+      P.part_col = o.part_col;
+      if (P.out_mode != kOutPartial) {
+        const long esz = P.out_mode == kOutBf16 ? 2 : 4;
+        P.out = static_cast<char *>(o.out) + (long)n0 * o.ldy * esz;
+      }
+      const long a_rows = o.a_mn ? (long)o.heads * K : (long)o.heads * o.M;
+      const long a_cols = o.a_mn ? o.M : K;
+      if (!map2d(&tm[i], o.A, a_rows, a_cols, 64, o.a_mn ? 64 : 128)) return cudaErrorInvalidValue;
+    }
+    if (nops == 1) tm[1] = tm[0];
+    if (!map2d(&tx, X + (long)n0 * x_cols, nn, x_cols, 64, g.n_pad)) return cudaErrorInvalidValue;
+    if (g.stages < 2) return cudaErrorInvalidValue;
+    const size_t smem = (size_t)g.stages * stage_bytes + 256 + 1024;
+    gemm_sm100_kernel<<<tiles, kThreads, smem, s>>>(tm[0], tm[1], tx, g);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t gemm_reduce(const float *part, int splits, int n, int width, int part_ld, void *out,
+                        long ldy, bool out_bf16, cudaStream_t s) {
+  const long total = (long)n * width;
+  int blocks = (int)((total + 255) / 256);
+  if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+  gemm_reduce_kernel<<<blocks, 256, 0, s>>>(part, splits, n, width, part_ld, out, ldy,
+                                            out_bf16 ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace sm100
+}  // namespace mla

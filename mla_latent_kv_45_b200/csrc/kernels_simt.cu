@@ -91,10 +91,6 @@ cudaError_t launch_gemv(const GemvArgs &a, int heads, cudaStream_t s) {
 #define MLA_INST_GEMV(TW, TX, TY) \
   template cudaError_t launch_gemv<TW, TX, TY>(const GemvArgs &, int, cudaStream_t);
 MLA_INST_GEMV(float, float, float)
-MLA_INST_GEMV(__nv_bfloat16, __nv_bfloat16, float)
-MLA_INST_GEMV(__nv_bfloat16, float, float)
-MLA_INST_GEMV(__nv_bfloat16, float, __nv_bfloat16)
-MLA_INST_GEMV(__nv_bfloat16, __nv_bfloat16, __nv_bfloat16)
 
 // ---------------------------------------------------------------------------
 // Cache-append epilogue: RMSNorm on c, RoPE on k_R, one rounding, paged write

@@ -186,7 +186,7 @@ mla_status mla_cache_append(const mla_dims *dims, const mla_paged_cache *cache, 
   }
   MLA_TRY(cuda_ok(sm100::append_proj(static_cast<const bf16 *>(h), static_cast<const bf16 *>(W_DKV),
                                      static_cast<const bf16 *>(W_KR), batch, d_model, xkv,
-                                     at(ws, L.gemm), s)));
+                                     at(ws, L.gemm), err, s)));
   return cuda_ok(launch_append_finish<bf16>(
       xkv, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
       static_cast<bf16 *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
@@ -238,10 +238,12 @@ mla_status mla_absorb_q(const mla_dims *dims, int batch, int d_in, const void *x
     return cuda_ok(launch_rope_q<float>(qr, batch, H, d.d_c, rp, positions,
                                         static_cast<float *>(q_lat), s));
   }
-  MLA_TRY(cuda_ok(sm100::absorb_proj(static_cast<const bf16 *>(x), static_cast<const bf16 *>(W_DQ),
-                                     static_cast<const bf16 *>(W_UQ), static_cast<const bf16 *>(W_QR),
-                                     static_cast<const bf16 *>(W_UK), batch, d_in, d_q, cq, qc, qr,
-                                     static_cast<bf16 *>(q_lat), at(ws, L.gemm), s)));
+  MLA_TRY(cuda_ok(sm100::absorb_proj(
+      static_cast<const bf16 *>(x), static_cast<const bf16 *>(W_DQ),
+      static_cast<const bf16 *>(W_UQ), static_cast<const bf16 *>(W_QR),
+      static_cast<const bf16 *>(W_UK), batch, d_in, d_q, reinterpret_cast<bf16 *>(cq),
+      reinterpret_cast<bf16 *>(qc), qr, static_cast<bf16 *>(q_lat), at(ws, L.gemm),
+      reinterpret_cast<int *>(at(ws, L.err)), s)));
   return cuda_ok(launch_rope_q<bf16>(qr, batch, H, d.d_c, rp, positions,
                                      static_cast<bf16 *>(q_lat), s));
 }
@@ -330,9 +332,10 @@ mla_status mla_unabsorb_out(const mla_dims *dims, int batch, const void *z, cons
     return gemv<float, float, float>(W_O, 0, (long)H * d.d_v, 1, o, 0, (long)H * d.d_v, out, 0,
                                      d_model, d_model, H * d.d_v, batch, 1, s);
   }
-  return cuda_ok(sm100::unabsorb_proj(static_cast<const bf16 *>(z), static_cast<const bf16 *>(W_UV),
-                                      static_cast<const bf16 *>(W_O), batch, d_model, o,
-                                      static_cast<bf16 *>(out), at(ws, L.gemm), s));
+  return cuda_ok(sm100::unabsorb_proj(
+      static_cast<const bf16 *>(z), static_cast<const bf16 *>(W_UV), static_cast<const bf16 *>(W_O),
+      batch, d_model, reinterpret_cast<bf16 *>(o), static_cast<bf16 *>(out), at(ws, L.gemm),
+      reinterpret_cast<int *>(at(ws, L.err)), s));
 }
 
 mla_status mla_get_device_error(void *ws, mla_stream_t stream) {

@@ -22,19 +22,20 @@ size_t gemm_workspace_bytes(int batch, int d_model, int d_q, int n_heads, const 
 // xkv[b] = [W_DKV h_b ; W_KR h_b] in fp32 ([batch][576]).
 cudaError_t append_proj(const __nv_bfloat16 *h, const __nv_bfloat16 *W_DKV,
                         const __nv_bfloat16 *W_KR, int batch, int d_model, float *xkv,
-                        void *gemm_ws, cudaStream_t s);
+                        void *gemm_ws, int *err, cudaStream_t s);
 
-// c_Q (fp32, when W_DQ), q_C (fp32), raw q_R (fp32, not yet rotated) and the
+// c_Q (bf16, when W_DQ), q_C (bf16), raw q_R (fp32, not yet rotated) and the
 // absorbed content half q_lat[b][i][0:512] = W_UK,i^T q_C,i (bf16).
 cudaError_t absorb_proj(const __nv_bfloat16 *x, const __nv_bfloat16 *W_DQ,
                         const __nv_bfloat16 *W_UQ, const __nv_bfloat16 *W_QR,
-                        const __nv_bfloat16 *W_UK, int batch, int d_in, int d_q, float *cq,
-                        float *qc, float *qr, __nv_bfloat16 *q_lat, void *gemm_ws, cudaStream_t s);
+                        const __nv_bfloat16 *W_UK, int batch, int d_in, int d_q,
+                        __nv_bfloat16 *cq, __nv_bfloat16 *qc, float *qr, __nv_bfloat16 *q_lat,
+                        void *gemm_ws, int *err, cudaStream_t s);
 
-// o[b][i] = W_UV,i z[b][i]; out = W_O o when W_O is given (o kept in fp32), else out = o.
+// o[b][i] = W_UV,i z[b][i] (bf16); out = W_O o when W_O is given, else out = o.
 cudaError_t unabsorb_proj(const __nv_bfloat16 *z, const __nv_bfloat16 *W_UV,
-                          const __nv_bfloat16 *W_O, int batch, int d_model, float *o,
-                          __nv_bfloat16 *out, void *gemm_ws, cudaStream_t s);
+                          const __nv_bfloat16 *W_O, int batch, int d_model, __nv_bfloat16 *o,
+                          __nv_bfloat16 *out, void *gemm_ws, int *err, cudaStream_t s);
 
 // Latent attention over the plan's partitions (partials / z / lse).
 cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s);
