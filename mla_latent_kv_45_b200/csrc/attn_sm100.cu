@@ -10,28 +10,28 @@
 //
 // Design (one CTA pair = a 2-CTA cluster per work partition):
 //  * The fp32 accumulator O = 128 x 512 would fill all 512 TMEM columns, so
-//    CTA r owns latent columns [256 r, 256 r + 256) of O and loads only its
-//    half of each page plus half of the k_R columns (288 of the 576 columns):
-//    every cached byte crosses HBM once.
-//  * TMEM per CTA: O half (256 columns), the CTA's 288-column slice of q_lat
-//    as the A operand of the score MMA (144 columns, bf16 pairs), S (64).
-//    Keeping q_lat in TMEM leaves shared memory for a 4-stage TMA ring.
-//  * Each CTA computes a partial score over its 288 columns (tcgen05.mma,
-//    M = 128 heads, N = 64 rows, K = 288) and writes it with asynchronous
-//    remote stores (st.async) into one of two receive slots in its partner's
-//    shared memory; each store completes bytes of the slot's mbarrier, so no
-//    thread fences or waits for its stores.  The exchange runs one tile
-//    ahead: the partial of tile j+1 is sent before tile j's softmax.  Both
-//    CTAs add the halves in the same order and run the identical online
-//    softmax (exp2 domain, lazy rescale when the max grows by more than 2^8).
-//  * Two softmax warpgroups: TMEM lane = head, warpgroup g owns the 32 rows
-//    [32 g, 32 g + 32) of each page; row maxima and sums are combined through
-//    shared memory.
-//  * P (bf16) goes to TMEM; O_half += P . V_half on tcgen05 with A = P read
-//    from TMEM and B = the page's latent half (N = 256).
-//  * Warp roles: warps 0-7 softmax + epilogue + q_lat staging, warp 8 TMA
-//    producer, warp 9 TMEM allocation + score MMA issue, warp 10 P.V MMA issue
-//    (two issuers, so P.V of tile j never waits for the data of tile j+1).
+//    CTA r owns latent columns [256 r, 256 r + 256) of O.
+//  * Rows of each 64-row page are split between the pair: CTA r scores its
+//    own 32 rows [32 r, 32 r + 32) over all 576 columns (tcgen05.mma,
+//    M = 128 heads, N = 32 rows, K = 576), so no partial score is exchanged.
+//    q_lat is the A operand: 448 of its columns sit in TMEM, the last 128
+//    (latent 448..511 and k_R) in shared memory.
+//  * Each CTA turns its own rows into P (bf16, exp2 domain) relative to a
+//    reference max that both CTAs share, and sends its P half plus the
+//    reference it used to the partner with st.async stores (8.5 KB per tile,
+//    counted by the receiving mbarrier).  When a CTA's own max grew past the
+//    shared reference by more than 2^8 it uses its own max instead; both CTAs
+//    then see the same pair of references, take the same new shared max,
+//    rescale O (TMEM) and the lagging P half (shared memory) identically.
+//  * O_half += P . V_half on tcgen05 (A = the 64-row P tile in shared
+//    memory, B = the page's latent half: the CTA's own rows come with its
+//    full-width tile, the partner's 32 rows are loaded separately and are
+//    normally L2 hits because the partner streams the same page).
+//  * Row sums are taken from the bf16 P both CTAs feed the MMA (own and
+//    received halves), so no sum is exchanged; the epilogue divides O_half.
+//  * Two softmax warpgroups (TMEM lane = head): warpgroup g owns 16 of the
+//    CTA's 32 rows.  Warp 8: TMA producer; warp 9: TMEM allocation + score
+//    MMAs + q_lat shared-memory part; warp 10: P.V MMAs.
 //  * Partitions come from the plan kernel (equal page counts); a sequence cut
 //    by a partition boundary writes an unnormalised partial that the combine
 //    kernel merges.
@@ -53,37 +53,45 @@ constexpr int kHeads = 128;
 constexpr int kRow = 576;        // cached values per row
 constexpr int kDc = 512;
 constexpr int kPage = 64;
-constexpr int kHalf = 256;       // latent columns per CTA
-constexpr int kStages = 4;
+constexpr int kOwn = 32;         // rows of a page scored by each CTA
+constexpr int kHalf = 256;       // latent columns of O per CTA
+constexpr int kStages = 3;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 96;   // + producer, score issuer, P.V issuer
 constexpr int kWarpProd = 8, kWarpS = 9, kWarpPV = 10;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Shared memory (byte offsets from a 1024-byte aligned base).
-constexpr int kKChunk = kPage * 128;             // 64 rows x 64 bf16, 128B swizzle
-constexpr int kKRope = kPage * 64;               // 64 rows x 32 bf16, 64B swizzle
-constexpr int kStageBytes = 4 * kKChunk + kKRope;  // 36 KB
-constexpr int kXBytes = 128 * 64 * 4;            // one partial-score tile (fp32)
-constexpr int kOffStage = 0;
-constexpr int kOffX = kOffStage + kStages * kStageBytes;  // two receive slots (partner's partials)
-constexpr int kOffRed = kOffX + 2 * kXBytes;     // 2 x 128 floats: per-warpgroup row max / sum
+constexpr int kChunk = kOwn * 128;               // 32 rows x 64 bf16, 128-byte swizzle
+constexpr int kQChunk = kHeads * 128;            // 128 heads x 64 bf16
+constexpr int kOffQ = 0;                         // q_lat columns 448..575 (2 chunks)
+constexpr int kOffStage = kOffQ + 2 * kQChunk;
+constexpr int kRegionB = 9 * kChunk;             // own rows: 9 chunks x 64 columns
+constexpr int kStageBytes = kRegionB + 4 * kChunk;  // + partner rows, own latent half
+constexpr int kPBytes = kHeads * 128;            // P tile: 128 heads x 64 rows bf16
+constexpr int kOffP = kOffStage + kStages * kStageBytes;   // two P tiles
+constexpr int kOffRef = kOffP + 2 * kPBytes;     // two x 128 received reference maxima
+constexpr int kOffRed = kOffRef + 1024;          // 2 x 128 floats: per-warpgroup scratch
 constexpr int kOffBar = kOffRed + 1024;
-constexpr int kSmemBytes = kOffBar + 256 + 1024;
+constexpr int kSmemBytes = kOffBar + 512 + 1024;
+constexpr uint32_t kMsgBytes = kHeads * kOwn * 2 + kHeads * 4;   // P half + references
 
 // TMEM columns
 constexpr uint32_t kTmemO = 0;     // O_half: 256 fp32 columns
-constexpr uint32_t kTmemQ = 256;   // q_lat slice: 288 bf16 = 144 columns
-constexpr uint32_t kTmemP = 400;   // P: 64 bf16 = 32 columns
-constexpr uint32_t kTmemS = 448;   // S: 64 fp32 columns
+constexpr uint32_t kTmemQ = 256;   // q_lat columns 0..447: 224 columns of bf16 pairs
+constexpr uint32_t kTmemS = 480;   // S: 32 fp32 columns
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0, 0);    // A = q_lat (TMEM), B = rows (K-major)
-constexpr uint32_t kIdescPV = idesc_bf16(128, 256, 0, 1);  // A = P (TMEM), B = V (MN-major)
+constexpr uint32_t kIdescS = idesc_bf16(128, kOwn, 0, 0);  // A = q_lat, B = own rows (K-major)
+constexpr uint32_t kIdescPV = idesc_bf16(128, 256, 0, 1);  // A = P (K-major), B = V (MN-major)
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_full, s_full, s_free, p_full, pv_done, x_full[2], peer_free[2], drain_s, drain_pv;
+  uint64_t q_tmem, q_smem, q_free, s_full, s_free, drain_s, drain_pv;
+  uint64_t pv_done[2];     // P.V of the tile using P tile slot i completed
+  uint64_t p_ready[2];     // own P half written and partner half final (8 softmax warps)
+  uint64_t p_rx[2];        // partner's P half + references landed (tx count)
+  uint64_t p_slot_free[2]; // partner's P tile slot may be overwritten (remote arrive)
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -115,6 +123,28 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t *>(&v);
 }
 
+// Sum of the 8 bf16 values in a 16-byte chunk, each scaled by f.
+__device__ __forceinline__ float sum8_bf16(uint4 v) {
+  const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&v);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(p[i]);
+    s += f.x + f.y;
+  }
+  return s;
+}
+
+__device__ __forceinline__ uint4 scale8_bf16(uint4 v, float f) {
+  __nv_bfloat162 *p = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(p[i]);
+    p[i] = __floats2bfloat162_rn(x.x * f, x.y * f);
+  }
+  return v;
+}
+
 // Named barrier over the 256 softmax threads.
 __device__ __forceinline__ void softmax_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
@@ -143,41 +173,27 @@ struct TileCursor {
   __device__ __forceinline__ bool last() const { return lp == seg.lp1 - 1; }
 };
 
-// Stages this warpgroup's share of the CTA's 288-column slice of q_lat[b][h]
-// into TMEM (lane h): warpgroup 0 the latent columns [0, 128) of the slice,
-// warpgroup 1 the latent columns [128, 256) and the 32 RoPE columns.
-__device__ __forceinline__ void stage_q(const AttnArgs &a, int b, int h, int g, uint32_t rank,
-                                        uint32_t taddr) {
+// Stages q_lat[b][h][0:448] into TMEM lane h (224 columns of bf16 pairs);
+// warpgroup 0 writes columns [0, 128), warpgroup 1 columns [128, 224).
+__device__ __forceinline__ void stage_q(const AttnArgs &a, int b, int h, int g, uint32_t taddr) {
   const uint4 *src = reinterpret_cast<const uint4 *>(
       reinterpret_cast<const __nv_bfloat16 *>(a.q_lat) + ((long)b * kHeads + h) * kRow);
-  const int c0 = kHalf * rank / 8;          // 16-byte units
-#pragma unroll
-  for (int blk = 0; blk < 2; ++blk) {       // 2 x 32 TMEM columns (64 bf16 each)
-    const int bb = 2 * g + blk;
+  const int b0 = g ? 4 : 0, b1 = g ? 7 : 4;       // blocks of 32 TMEM columns
+  for (int bb = b0; bb < b1; ++bb) {
     uint32_t v[32];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint4 x = src[c0 + bb * 8 + i];
+      const uint4 x = src[bb * 8 + i];
       v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
     }
     tmem_st32(taddr + 32 * bb, v);
-  }
-  if (g == 1) {                             // RoPE part: 16 TMEM columns
-    const int r0 = (kDc + 32 * rank) / 8;
-    uint32_t w[16];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 x = src[r0 + i];
-      w[4 * i] = x.x; w[4 * i + 1] = x.y; w[4 * i + 2] = x.z; w[4 * i + 3] = x.w;
-    }
-    tmem_st16(taddr + 128, w);
   }
   tmem_wait_st();
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_kv,
-                      const __grid_constant__ CUtensorMap tm_kr, const AttnArgs a,
+                      const __grid_constant__ CUtensorMap tm_q, const AttnArgs a,
                       const float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -195,26 +211,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->q_full, 8);
+    mbar_init(&bars->q_tmem, 8);
+    mbar_init(&bars->q_smem, 1);
+    mbar_init(&bars->q_free, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 8);
-    mbar_init(&bars->p_full, 8);
-    mbar_init(&bars->pv_done, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->x_full[i], 1);
-      mbar_init(&bars->peer_free[i], 1);
-    }
     mbar_init(&bars->drain_s, 1);
     mbar_init(&bars->drain_pv, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->pv_done[i], 1);
+      mbar_init(&bars->p_ready[i], 8);
+      mbar_init(&bars->p_rx[i], 1);
+      mbar_init(&bars->p_slot_free[i], 1);
+    }
     bars->abort = 0;
     fence_mbar_init();
     // arm both receive slots for tiles 0 and 1 before the partner can send
-    mbar_expect_tx(&bars->x_full[0], kXBytes);
-    mbar_expect_tx(&bars->x_full[1], kXBytes);
+    mbar_expect_tx(&bars->p_rx[0], kMsgBytes);
+    mbar_expect_tx(&bars->p_rx[1], kMsgBytes);
   }
   if (warp == kWarpProd && lane == 0) {
     prefetch_tmap(&tm_kv);
-    prefetch_tmap(&tm_kr);
+    prefetch_tmap(&tm_q);
   }
   if (warp == kWarpS) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -222,7 +240,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   tc_fence_after();
-  cluster_sync();  // the partner's barriers exist before any remote arrive or copy
+  cluster_sync();  // the partner's barriers exist (and are armed) before any remote access
   const uint32_t tmem = bars->tmem_base;
 
   TileCursor cur;
@@ -245,57 +263,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         uint8_t *dst = smem + kOffStage + st * kStageBytes;
         mbar_expect_tx(&bars->full[st], kStageBytes);
-        const int y = page * kPage;
-        for (int i = 0; i < 4; ++i)
-          tma_load_2d(dst + i * kKChunk, &tm_kv, kHalf * rank + 64 * i, y, &bars->full[st]);
-        tma_load_2d(dst + 4 * kKChunk, &tm_kr, kDc + 32 * rank, y, &bars->full[st]);
+        const int y_own = page * kPage + kOwn * rank;
+        const int y_peer = page * kPage + kOwn * (1 - rank);
+        for (int c = 0; c < 9; ++c)        // own rows, all 576 columns
+          tma_load_2d(dst + c * kChunk, &tm_kv, 64 * c, y_own, &bars->full[st]);
+        for (int c = 0; c < 4; ++c)        // partner rows, this CTA's latent half
+          tma_load_2d(dst + kRegionB + c * kChunk, &tm_kv, kHalf * rank + 64 * c, y_peer,
+                      &bars->full[st]);
       }
-      // drain: every issued load lands before the CTA may exit
       for (int t = tile - kStages; t < tile; ++t)
         if (t >= 0) wait_bar<false>(ctx, &bars->full[t % kStages], (t / kStages) & 1);
     }
   } else if (warp == kWarpS) {
-    // ------------------------------------------------------------ score MMA issuer
+    // ---------------------------------------- score MMA issuer (+ q_lat smem part)
     if (lane == 0) {
+      const uint32_t q_base = smem_u32(smem + kOffQ);
       int tile = 0;
+      bool ok = true;
       for (; cur.valid; cur.advance(a), ++tile) {
         const int st = tile % kStages;
-        if (!wait_bar<false>(ctx, &bars->full[st], (tile / kStages) & 1)) break;
-        if (cur.first() && !wait_bar<false>(ctx, &bars->q_full, cur.nseg & 1)) break;
-        if (tile > 0 && !wait_bar<false>(ctx, &bars->s_free, (tile - 1) & 1)) break;
+        if (cur.first()) {
+          // the previous segment's score MMAs must finish before q_lat is replaced
+          if (cur.nseg > 0 && !wait_bar<false>(ctx, &bars->q_free, (cur.nseg - 1) & 1)) { ok = false; break; }
+          mbar_expect_tx(&bars->q_smem, 2 * kQChunk);
+          tma_load_2d(smem + kOffQ, &tm_q, 448, cur.seg.b * kHeads, &bars->q_smem);
+          tma_load_2d(smem + kOffQ + kQChunk, &tm_q, 512, cur.seg.b * kHeads, &bars->q_smem);
+          if (!wait_bar<false>(ctx, &bars->q_smem, cur.nseg & 1)) { ok = false; break; }
+          if (!wait_bar<false>(ctx, &bars->q_tmem, cur.nseg & 1)) { ok = false; break; }
+        }
+        if (!wait_bar<false>(ctx, &bars->full[st], (tile / kStages) & 1)) { ok = false; break; }
+        if (tile > 0 && !wait_bar<false>(ctx, &bars->s_free, (tile - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t k_base = smem_u32(smem + kOffStage + st * kStageBytes);
-        int kk = 0;
-        for (int i = 0; i < 4; ++i)         // latent columns: 4 chunks of 64, 128B swizzle
-          for (int k = 0; k < 4; ++k, ++kk)
-            umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 32 * i + 8 * k,
-                         sdesc(k_base + i * kKChunk + 32 * k, 16, 1024, 2), kIdescS,
-                         kk ? 1u : 0u);
-        for (int k = 0; k < 2; ++k)         // RoPE columns: 32 wide, 64B swizzle
-          umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 128 + 8 * k,
-                       sdesc(k_base + 4 * kKChunk + 32 * k, 16, 512, 4), kIdescS, 1u);
+        for (int s = 0; s < 28; ++s)        // q_lat columns 0..447 from TMEM
+          umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * s,
+                       sdesc(k_base + (s >> 2) * kChunk + 32 * (s & 3), 16, 1024, 2), kIdescS,
+                       s ? 1u : 0u);
+        for (int s = 0; s < 8; ++s)         // columns 448..575 from shared memory
+          umma_bf16(tmem + kTmemS, sdesc(q_base + (s >> 2) * kQChunk + 32 * (s & 3), 16, 1024, 2),
+                    sdesc(k_base + (7 + (s >> 2)) * kChunk + 32 * (s & 3), 16, 1024, 2), kIdescS,
+                    1u);
+        if (cur.last()) umma_commit(&bars->q_free);
         umma_commit(&bars->s_full);
       }
+      (void)ok;
       umma_commit(&bars->drain_s);
       wait_bar<false>(ctx, &bars->drain_s, 0);
     }
   } else if (warp == kWarpPV) {
     // ------------------------------------------------------------ P.V MMA issuer
     if (lane == 0) {
+      const uint32_t p_base = smem_u32(smem + kOffP);
       int tile = 0;
       for (; cur.valid; cur.advance(a), ++tile) {
         const int st = tile % kStages;
-        if (!wait_bar<false>(ctx, &bars->p_full, tile & 1)) break;
+        const int pb = tile & 1;
+        if (!wait_bar<false>(ctx, &bars->p_ready[pb], (tile >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + kOffStage + st * kStageBytes);
         const bool first = cur.first();
-        for (int k = 0; k < kPage / 16; ++k)
-          // A: P rows (heads) x 16 tokens (TMEM, 8 columns per step); B: 16 tokens
-          // x 256 latent (MN-major, 64-column chunks 8 KB apart, 8-token groups 1 KB apart)
-          umma_bf16_ts(tmem + kTmemO, tmem + kTmemP + 8 * k,
-                       sdesc(v_base + 2048 * k, kKChunk, 1024, 2), kIdescPV,
-                       (first && k == 0) ? 0u : 1u);
-        umma_commit(&bars->pv_done);
+        for (int k = 0; k < kPage / 16; ++k) {
+          // rows [16 k, 16 k + 16) of the page: own rows (full-width tile, latent
+          // half = chunks 4r..4r+3) or partner rows (region B); chunks 4 KB apart
+          const bool own = (k >> 1) == (int)rank;
+          const uint32_t vb = v_base + (own ? 4 * rank * kChunk : kRegionB) + (k & 1) * 2048;
+          umma_bf16(tmem + kTmemO, sdesc(p_base + pb * kPBytes + 32 * k, 16, 1024, 2),
+                    sdesc(vb, kChunk, 1024, 2), kIdescPV, (first && k == 0) ? 0u : 1u);
+        }
+        umma_commit(&bars->pv_done[pb]);
         umma_commit(&bars->empty[st]);
       }
       umma_commit(&bars->drain_pv);
@@ -303,109 +338,135 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ----------------------- softmax + epilogue + q_lat staging (warps 0-7)
-    const int g = warp >> 2;                 // warpgroup: rows [32 g, 32 g + 32) of a page
+    const int g = warp >> 2;                 // warpgroup: own rows [16 g, 16 g + 16)
     const int h = threadIdx.x & 127;         // head index == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float *red = reinterpret_cast<float *>(smem + kOffRed);   // [2][128]
-    // partial-score tile layout (per receive slot): 16-byte chunk i (4 rows of a
-    // page) of head h at (i * 128 + h) * 16; warpgroup g owns chunks [8 g, 8 g + 8)
-    const uint32_t x_local = smem_u32(smem + kOffX) + h * 16;
-    const uint32_t x_remote = mapa(x_local, peer);
-    const uint32_t peer_x_full = mapa(smem_u32(&bars->x_full[0]), peer);
-    const uint32_t peer_free = mapa(smem_u32(&bars->peer_free[0]), peer);
-    TileCursor nxt = cur;
-    float m_run = -INFINITY, l_part = 0.f;
-    int tile = 0;
-    float sa[32], sb[32];
+    const float *refs = reinterpret_cast<const float *>(smem + kOffRef);  // [2][128]
+    uint8_t *pt = smem + kOffP;
+    // P tile row h: 16-byte chunk c (rows 8c..8c+7 of the page) at h*128 + ((c ^ (h&7)) << 4)
+    const int c_own = 4 * rank + 2 * g;      // this thread's two own chunks: c_own, c_own + 1
+    const int c_peer = 4 * (1 - rank) + 2 * g;  // and the matching partner chunks
+    const uint32_t p_local = smem_u32(pt) + h * 128;
+    const uint32_t p_remote = mapa(p_local, peer);
+    const uint32_t ref_remote = mapa(smem_u32(smem + kOffRef) + h * 4, peer);
+    const uint32_t rx_remote = mapa(smem_u32(&bars->p_rx[0]), peer);
+    const uint32_t slot_free_remote = mapa(smem_u32(&bars->p_slot_free[0]), peer);
 
-    // S_j: this warpgroup's 32 score columns from TMEM into s, then sent to
-    // the partner's receive slot j % 2 (its mbarrier counts the bytes)
-    auto fetch_and_store = [&](int j, float (&s)[32]) -> bool {
+    float m_run = -INFINITY;     // shared reference max (log2 units), same in both CTAs
+    float l_part = 0.f;          // this thread's share of the row sum (own + partner chunks)
+    float ref_own = -INFINITY;   // reference used for the latest own P half
+
+    // ---- tile j: own rows -> P half (local + partner), reference sent along
+    auto produce = [&](int j, const TileCursor &tc) -> bool {
+      if (tc.first()) {
+        // the previous segment's score MMAs have completed (their S was read)
+        stage_q(a, tc.seg.b, h, g, tmem + lane_off + kTmemQ);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_tmem);
+        m_run = -INFINITY;
+      }
       if (!wait_bar<false>(ctx, &bars->s_full, j & 1)) return false;
       tc_fence_after();
-      tmem_ld32f(tmem + lane_off + kTmemS + 32 * g, s);
+      float sv[16];
+      tmem_ld16f(tmem + lane_off + kTmemS + 16 * g, sv);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_free);
-      const int slot = j & 1;
-      if (j >= 2 && !wait_bar<true>(ctx, &bars->peer_free[slot], ((j >> 1) - 1) & 1)) return false;
-      const uint32_t dst = x_remote + slot * kXBytes;
-      const uint32_t mb = peer_x_full + slot * 8;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        st_async_v4(dst + (8 * g + i) * 2048, s[4 * i], s[4 * i + 1], s[4 * i + 2], s[4 * i + 3],
-                    mb);
-      return true;
-    };
-    auto stage_segment_q = [&](int b) {
-      stage_q(a, b, h, g, rank, tmem + lane_off + kTmemQ);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->q_full);
-    };
-
-    bool ok = cur.valid;
-    if (ok) {
-      stage_segment_q(cur.seg.b);
-      ok = fetch_and_store(0, sa);
-      nxt.advance(a);
-    }
-    // One tile: look ahead (stage q_lat of the next segment, fetch and store
-    // S_{j+1} from `sn`), combine S_j (in `sc`) with the partner's partial,
-    // softmax, P, release S_{j+1}, and the epilogue at the end of a segment.
-    auto step = [&](float (&sc)[32], float (&sn)[32]) -> bool {
-      const bool ahead = nxt.valid;
-      if (ahead) {
-        // S_j, the last score MMA that read the old q_lat, is complete
-        if (nxt.first()) stage_segment_q(nxt.seg.b);
-        if (!fetch_and_store(tile + 1, sn)) return false;
-      }
-      // ---- combine tile j with the partner's partial
-      const int slot = tile & 1;
-      if (!wait_bar<true>(ctx, &bars->x_full[slot], (tile >> 1) & 1)) return false;
-      const bool first = cur.first();
-      if (first) {
-        m_run = -INFINITY;
-        l_part = 0.f;
-      }
-      const uint8_t *xr = smem + kOffX + slot * kXBytes + h * 16;
+      const int rows_valid = tc.seg.len - tc.lp * kPage;          // >= 1
+      const int own_valid = min(max(rows_valid - kOwn * (int)rank, 0), kOwn);
+      const int mine = own_valid - 16 * g;                          // valid among my 16
       float mx = -INFINITY;
-      const int n_valid = min(kPage, cur.seg.len - cur.lp * kPage);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 v = *reinterpret_cast<const float4 *>(xr + (8 * g + i) * 2048);
-        // rank 0 adds (own + partner), rank 1 (partner + own): the same sum
-        if (rank == 0) {
-          sc[4 * i] += v.x; sc[4 * i + 1] += v.y; sc[4 * i + 2] += v.z; sc[4 * i + 3] += v.w;
-        } else {
-          sc[4 * i] = v.x + sc[4 * i]; sc[4 * i + 1] = v.y + sc[4 * i + 1];
-          sc[4 * i + 2] = v.z + sc[4 * i + 2]; sc[4 * i + 3] = v.w + sc[4 * i + 3];
+      for (int k = 0; k < 16; ++k) {
+        sv[k] = k < mine ? sv[k] : -INFINITY;
+        mx = fmaxf(mx, sv[k]);
+      }
+      softmax_sync();                        // previous readers of red[] are done
+      red[g * 128 + h] = mx;
+      softmax_sync();
+      const float mx_own = fmaxf(red[h], red[128 + h]) * scale_log2;
+      ref_own = (mx_own > m_run + 8.0f) ? mx_own : m_run;
+      uint32_t w[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float p0 = 2 * q < mine ? ex2(fmaf(sv[2 * q], scale_log2, -ref_own)) : 0.f;
+        const float p1 = 2 * q + 1 < mine ? ex2(fmaf(sv[2 * q + 1], scale_log2, -ref_own)) : 0.f;
+        w[q] = pack_bf16(p0, p1);
+      }
+      // rows past the sequence end hold arbitrary bytes: zero their latent
+      // half in the stage so that 0 * garbage cannot reach O
+      if (rows_valid < kPage) {
+        uint8_t *stg = smem + kOffStage + (j % kStages) * kStageBytes;
+        const int peer_valid = min(max(rows_valid - kOwn * (1 - (int)rank), 0), kOwn);
+        for (int i = threadIdx.x; i < 2 * kOwn * 32; i += kSoftmaxThreads) {
+          const int piece = i & 31, row = (i >> 5) % kOwn, which = i >> 10;
+          const int valid = which ? peer_valid : own_valid;
+          if (row >= valid) {
+            uint8_t *base = which ? stg + kRegionB : stg + 4 * rank * kChunk;
+            *reinterpret_cast<uint4 *>(base + (piece >> 3) * kChunk + row * 128 +
+                                       (piece & 7) * 16) = make_uint4(0, 0, 0, 0);
+          }
         }
       }
-#pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        sc[k] = 32 * g + k < n_valid ? sc[k] : -INFINITY;
-        mx = fmaxf(mx, sc[k]);
+      const int pb = j & 1;
+      if (j >= 2) {
+        // this CTA's P.V of tile j-2 read P tile pb: free it locally and for the partner
+        if (!wait_bar<false>(ctx, &bars->pv_done[pb], ((j >> 1) - 1) & 1)) return false;
+        if (threadIdx.x == 0) mbar_arrive_cluster_relaxed(slot_free_remote + pb * 8);
+        if (!wait_bar<true>(ctx, &bars->p_slot_free[pb], ((j >> 1) - 1) & 1)) return false;
       }
-      red[g * 128 + h] = mx;
-      softmax_sync();                        // slot read by all: the partner may refill it
-      if (threadIdx.x == 0) {
-        mbar_expect_tx(&bars->x_full[slot], kXBytes);   // armed for tile j + 2
-        mbar_arrive_cluster_relaxed(peer_free + slot * 8);
+      const uint4 v0 = make_uint4(w[0], w[1], w[2], w[3]);
+      const uint4 v1 = make_uint4(w[4], w[5], w[6], w[7]);
+      const uint32_t o0 = pb * kPBytes + ((c_own ^ (h & 7)) << 4);
+      const uint32_t o1 = pb * kPBytes + (((c_own + 1) ^ (h & 7)) << 4);
+      *reinterpret_cast<uint4 *>(pt + h * 128 + o0) = v0;
+      *reinterpret_cast<uint4 *>(pt + h * 128 + o1) = v1;
+      const uint32_t mb = rx_remote + pb * 8;
+      st_async_v4u(p_remote + o0, v0, mb);
+      st_async_v4u(p_remote + o1, v1, mb);
+      if (g == 0) st_async_f32(ref_remote + pb * 512, ref_own, mb);
+      return true;
+    };
+
+    // ---- tile j: the partner's half and reference have landed: shared max,
+    // rescales, row sums; hand the P tile to the P.V issuer
+    auto finalize = [&](int j, const TileCursor &tc) -> bool {
+      const int pb = j & 1;
+      if (!wait_bar<true>(ctx, &bars->p_rx[pb], (j >> 1) & 1)) return false;
+      if (threadIdx.x == 0) mbar_expect_tx(&bars->p_rx[pb], kMsgBytes);   // armed for tile j + 2
+      const float ref_p = refs[pb * 128 + h];
+      const float m_new = fmaxf(ref_own, ref_p);
+      const bool first = tc.first();
+      const float f_own = ref_own < m_new ? ex2(ref_own - m_new) : 1.f;
+      const float f_peer = ref_p < m_new ? ex2(ref_p - m_new) : 1.f;
+      const float alpha = (first || !(m_new > m_run)) ? 1.f : ex2(m_run - m_new);
+      uint8_t *row = pt + pb * kPBytes + h * 128;
+      uint4 *q0 = reinterpret_cast<uint4 *>(row + ((c_own ^ (h & 7)) << 4));
+      uint4 *q1 = reinterpret_cast<uint4 *>(row + (((c_own + 1) ^ (h & 7)) << 4));
+      uint4 *q2 = reinterpret_cast<uint4 *>(row + ((c_peer ^ (h & 7)) << 4));
+      uint4 *q3 = reinterpret_cast<uint4 *>(row + (((c_peer + 1) ^ (h & 7)) << 4));
+      uint4 own0 = *q0, own1 = *q1, pe0 = *q2, pe1 = *q3;
+      if (f_own != 1.f) {                    // rare: this CTA's reference was the lower one
+        own0 = scale8_bf16(own0, f_own);
+        own1 = scale8_bf16(own1, f_own);
+        *q0 = own0;
+        *q1 = own1;
       }
-      mx = fmaxf(mx, red[(g ^ 1) * 128 + h]) * scale_log2;
-      // ---- online softmax in the exp2 domain (identical in both warpgroups)
-      const bool grow = mx > m_run + 8.0f;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m_run - mx);
-        m_run = mx;
+      if (f_peer != 1.f) {                   // rare: the partner's reference was the lower one
+        pe0 = scale8_bf16(pe0, f_peer);
+        pe1 = scale8_bf16(pe1, f_peer);
+        *q2 = pe0;
+        *q3 = pe1;
       }
-      // P buffer and O are free once the previous tile's P.V has completed
-      if (tile > 0 && !wait_bar<false>(ctx, &bars->pv_done, (tile - 1) & 1)) return false;
-      tc_fence_after();
-      if (!first && __any_sync(0xffffffffu, grow)) {
+      const float add = (sum8_bf16(own0) + sum8_bf16(own1)) + (sum8_bf16(pe0) + sum8_bf16(pe1));
+      l_part = first ? add : l_part * alpha + add;
+      // O holds tiles < j of this segment; rescale it when the shared max moved
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!wait_bar<false>(ctx, &bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) return false;
+        tc_fence_after();
         for (int c = 128 * g; c < 128 * g + 128; c += 32) {
           uint32_t r[32];
           tmem_ld32(tmem + lane_off + kTmemO + c, r);
@@ -416,94 +477,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
       }
-      // P row h, rows [32 g, 32 g + 32) of the page: TMEM columns
-      // [16 g, 16 g + 16) of P, two bf16 per column (lower row in the low half)
-      float sum = 0.f;
-      {
-        uint32_t w[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float p0 = ex2(fmaf(sc[2 * q], scale_log2, -m_run));
-          const float p1 = ex2(fmaf(sc[2 * q + 1], scale_log2, -m_run));
-          sum += p0 + p1;
-          w[q] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tmem + lane_off + kTmemP + 16 * g, w);
-        tmem_wait_st();
-      }
-      l_part = l_part * alpha + sum;
-      if (n_valid < kPage) {
-        // rows past the sequence end hold arbitrary bytes: zero their latent
-        // part so that 0 * garbage cannot reach O
-        uint8_t *stg = smem + kOffStage + (tile % kStages) * kStageBytes;
-        const int nz = (kPage - n_valid) * 32;   // 16-byte pieces over 4 chunks
-        for (int i = threadIdx.x; i < nz; i += kSoftmaxThreads) {
-          const int row = n_valid + (i >> 5), piece = i & 31;
-          *reinterpret_cast<uint4 *>(stg + (piece >> 3) * kKChunk + row * 128 +
-                                     (piece & 7) * 16) = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
+      m_run = m_new;
+      fence_proxy_async_smem();              // own P, rescaled halves, zeroed rows -> MMA
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full);
-      if (cur.last()) {
-        // ---------------------------------------------------- epilogue
-        softmax_sync();                      // red[] reads of this tile are done
-        red[g * 128 + h] = l_part;
-        if (!wait_bar<false>(ctx, &bars->pv_done, tile & 1)) return false;
-        softmax_sync();
-        const float l_run = red[h] + red[128 + h];
-        softmax_sync();                      // red[] is free for the next tile's maxima
-        tc_fence_after();
-        const int pb = a.part_base[cur.seg.b];
-        const bool whole = pb < 0;
-        const long row_idx = (long)cur.seg.b * kHeads + h;
-        const int slot_p = whole ? 0 : pb + (part - cur.seg.s0 / hdr.quota);
-        const float inv_l = 1.f / l_run;
-        for (int c = 128 * g; c < 128 * g + 128; c += 32) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_off + kTmemO + c, r);
-          tmem_wait_ld();
-          if (whole) {
-            __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + row_idx * kDc +
-                               kHalf * rank + c;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(r[8 * j + 0]) * inv_l, __uint_as_float(r[8 * j + 1]) * inv_l);
-              v.y = pack_bf16(__uint_as_float(r[8 * j + 2]) * inv_l, __uint_as_float(r[8 * j + 3]) * inv_l);
-              v.z = pack_bf16(__uint_as_float(r[8 * j + 4]) * inv_l, __uint_as_float(r[8 * j + 5]) * inv_l);
-              v.w = pack_bf16(__uint_as_float(r[8 * j + 6]) * inv_l, __uint_as_float(r[8 * j + 7]) * inv_l);
-              *reinterpret_cast<uint4 *>(z + 8 * j) = v;
-            }
-          } else {
-            float *o = a.part_O + ((long)slot_p * kHeads + h) * kDc + kHalf * rank + c;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4 *>(o + 4 * j) =
-                  make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          }
-        }
-        if (rank == 0 && g == 0) {
-          const float ln2 = 0.6931471805599453f;
-          if (whole) {
-            if (a.lse) a.lse[row_idx] = (m_run + __log2f(l_run)) * ln2;
-          } else {
-            a.part_m[(long)slot_p * kHeads + h] = m_run * ln2;
-            a.part_l[(long)slot_p * kHeads + h] = l_run;
-          }
-        }
-        tc_fence_before();
-      }
-      cur.advance(a);
-      nxt.advance(a);
-      ++tile;
+      if (lane == 0) mbar_arrive(&bars->p_ready[pb]);
       return true;
     };
-    while (ok && cur.valid) {
-      if (!step(sa, sb)) break;
-      if (!cur.valid || !step(sb, sa)) break;
+
+    // ---- end of a segment (tile j was its last): normalise and write O_half
+    auto epilogue = [&](int j, const TileCursor &tc) -> bool {
+      softmax_sync();                        // previous readers of red[] are done
+      red[g * 128 + h] = l_part;
+      if (!wait_bar<false>(ctx, &bars->pv_done[j & 1], (j >> 1) & 1)) return false;
+      softmax_sync();
+      const float l_run = red[h] + red[128 + h];
+      tc_fence_after();
+      const int pbase = a.part_base[tc.seg.b];
+      const bool whole = pbase < 0;
+      const long row_idx = (long)tc.seg.b * kHeads + h;
+      const int slot_p = whole ? 0 : pbase + (part - tc.seg.s0 / hdr.quota);
+      const float inv_l = 1.f / l_run;
+      for (int c = 128 * g; c < 128 * g + 128; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + kTmemO + c, r);
+        tmem_wait_ld();
+        if (whole) {
+          __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + row_idx * kDc +
+                             kHalf * rank + c;
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint4 v;
+            v.x = pack_bf16(__uint_as_float(r[8 * jj + 0]) * inv_l, __uint_as_float(r[8 * jj + 1]) * inv_l);
+            v.y = pack_bf16(__uint_as_float(r[8 * jj + 2]) * inv_l, __uint_as_float(r[8 * jj + 3]) * inv_l);
+            v.z = pack_bf16(__uint_as_float(r[8 * jj + 4]) * inv_l, __uint_as_float(r[8 * jj + 5]) * inv_l);
+            v.w = pack_bf16(__uint_as_float(r[8 * jj + 6]) * inv_l, __uint_as_float(r[8 * jj + 7]) * inv_l);
+            *reinterpret_cast<uint4 *>(z + 8 * jj) = v;
+          }
+        } else {
+          float *o = a.part_O + ((long)slot_p * kHeads + h) * kDc + kHalf * rank + c;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj)
+            *reinterpret_cast<uint4 *>(o + 4 * jj) =
+                make_uint4(r[4 * jj], r[4 * jj + 1], r[4 * jj + 2], r[4 * jj + 3]);
+        }
+      }
+      if (rank == 0 && g == 0) {
+        const float ln2 = 0.6931471805599453f;
+        if (whole) {
+          if (a.lse) a.lse[row_idx] = (m_run + __log2f(l_run)) * ln2;
+        } else {
+          a.part_m[(long)slot_p * kHeads + h] = m_run * ln2;
+          a.part_l[(long)slot_p * kHeads + h] = l_run;
+        }
+      }
+      tc_fence_before();
+      return true;
+    };
+
+    TileCursor prev = cur;
+    bool ok = true;
+    for (int tile = 0; ok; ++tile) {
+      if (tile > 0) {
+        if (!finalize(tile - 1, prev)) break;
+        if (prev.last() && !epilogue(tile - 1, prev)) break;
+      }
+      if (!cur.valid) break;
+      if (!produce(tile, cur)) break;
+      prev = cur;
+      cur.advance(a);
     }
   }
 
@@ -559,13 +601,14 @@ cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  CUtensorMap tm_kv, tm_kr;
+  CUtensorMap tm_kv, tm_q;
   const long pool_rows = (long)a.num_pages * kPage;
-  if (!make_map(&tm_kv, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_kr, a.pool, pool_rows, 32, kPage, CU_TENSOR_MAP_SWIZZLE_64B))
+  const long q_rows = (long)a.batch * kHeads;
+  if (!make_map(&tm_kv, a.pool, pool_rows, 64, kOwn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm_q, a.q_lat, q_rows, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  attn_sm100_kernel<<<2 * parts, kThreads, kSmemBytes, s>>>(tm_kv, tm_kr, a, scale_log2);
+  attn_sm100_kernel<<<2 * parts, kThreads, kSmemBytes, s>>>(tm_kv, tm_q, a, scale_log2);
   return cudaGetLastError();
 }
 

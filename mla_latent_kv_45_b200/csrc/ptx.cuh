@@ -187,6 +187,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr));
 }
 
+// 16 consecutive TMEM columns of this thread's lane as fp32 (warp-collective).
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float *v) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+        "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]),
+        "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr));
+}
+
 // Same as tmem_ld32, delivering fp32 values straight into v[0..31].
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float *v) {
   asm volatile(
@@ -259,6 +270,19 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, flo
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
       ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(mbar)
       : "memory");
+}
+
+__device__ __forceinline__ void st_async_v4u(uint32_t addr, uint4 v, uint32_t mbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(mbar)
+      : "memory");
+}
+
+__device__ __forceinline__ void st_async_f32(uint32_t addr, float a, uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               ::"r"(addr), "r"(__float_as_uint(a)), "r"(mbar)
+               : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c,
