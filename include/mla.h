@@ -42,8 +42,8 @@
  *     positions outside the sequence's pages) skip the offending sequence (its
  *     outputs are zeroed, nothing is written out of bounds) and set the error
  *     word in the workspace; read it with mla_get_device_error().
- *   - Supported shapes: MLA_FP32 accepts any n_heads <= 256, d_c <= 1024,
- *     d_rope <= 128 (even), d_nope, d_v <= 256, page_size >= 1.  MLA_BF16
+ *   - Supported shapes: MLA_FP32 accepts any n_heads <= 256, d_c <= 1024 (a
+ *     multiple of 4), d_rope <= 128 (even), d_nope, d_v <= 256, page_size >= 1.  MLA_BF16
  *     requires the DeepSeek-V2 attention sizes n_heads = 128, d_c = 512,
  *     d_rope = 64, d_nope = d_v = 128, page_size = 64, and d_model, d_q
  *     multiples of 64; other shapes return MLA_ERR_UNSUPPORTED.

@@ -5,16 +5,19 @@
 // weight-bandwidth bound (each weight element is used B times), so the design
 // streams the weights once through a deep TMA ring with as many CTAs as it
 // takes to keep HBM busy:
-//  * each CTA owns one 128-row tile of one problem and a K range (split-K);
-//    D = A_tile . X^T accumulates in TMEM (tcgen05.mma, M = 128, N = batch
-//    padded to 16, K = 16 per instruction);
+//  * a work item is one 128-row tile of one problem, one K range (split-K) and
+//    one head; D = A_tile . X^T accumulates in TMEM (tcgen05.mma, M = 128,
+//    N = batch padded to 16, K = 16 per instruction);
+//  * CTAs are persistent over a contiguous range of items: the TMA ring runs
+//    on across items and the accumulator is double-buffered in TMEM, so one
+//    item's epilogue overlaps the next item's loads and MMAs;
 //  * A comes K-major ([out][in] weights) or MN-major (a per-head transposed
 //    view such as W_UK,i^T) -- both through 128-byte-swizzled TMA boxes;
 //  * X (the activations, bf16) is reloaded from L2 per K chunk;
-//  * several problems that share X (e.g. W_DKV and W_KR, W_UQ and W_QR) run
-//    in one launch; per-head problems (W_UK, W_UV) index heads in the grid;
+//  * two problems that share X (e.g. W_DKV and W_KR, W_UQ and W_QR) run in one
+//    launch; per-head problems (W_UK, W_UV) index heads in their items;
 //  * the epilogue writes bf16 / fp32 outputs directly or fp32 split-K
-//    partials that gemm_reduce sums in a fixed order (deterministic).
+//    partials that are summed in a fixed order (deterministic).
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue,
 // warps 2-5 epilogue.  Every wait is bounded (globaltimer).
 #include <cuda.h>
@@ -34,7 +37,7 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr int kABytes = 128 * 128;  // 128 rows x 64 bf16
 
 struct Bars {
-  uint64_t full[kMaxGemmStages], empty[kMaxGemmStages], d_full, drain;
+  uint64_t full[kMaxGemmStages], empty[kMaxGemmStages], acc_full[2], acc_free[2], drain;
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -54,6 +57,24 @@ __device__ __forceinline__ bool gwait(Bars *bars, int *err, uint64_t *bar, uint3
   }
 }
 
+struct Item {
+  int pi, head, split, m0, kc0, nk;
+};
+
+__device__ __forceinline__ Item decode_item(const GemmLaunch &g, int item) {
+  Item it;
+  it.pi = (g.nprob > 1 && item >= g.p[1].item_begin) ? 1 : 0;
+  const GemmProblem &P = g.p[it.pi];
+  int t = item - P.item_begin;
+  it.m0 = (t % P.m_tiles) * 128;
+  t /= P.m_tiles;
+  it.split = t % P.splits;
+  it.head = t / P.splits;
+  it.kc0 = it.split * P.chunks_per_split;
+  it.nk = min(g.k_chunks, it.kc0 + P.chunks_per_split) - it.kc0;
+  return it;
+}
+
 __global__ void __launch_bounds__(kThreads, 2)
     gemm_sm100_kernel(const __grid_constant__ CUtensorMap tm_a0,
                       const __grid_constant__ CUtensorMap tm_a1,
@@ -64,34 +85,25 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int stage_bytes = kABytes + g.n_pad * 128;
   Bars *bars = reinterpret_cast<Bars *>(smem + g.stages * stage_bytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // which problem / tile / split / head this CTA computes
-  int pi = 0;
-  while (pi + 1 < g.nprob && (int)blockIdx.x >= g.p[pi + 1].tile_begin) ++pi;
-  const GemmProblem &P = g.p[pi];
-  int t = blockIdx.x - P.tile_begin;
-  const int m_tile = t % P.m_tiles;
-  t /= P.m_tiles;
-  const int split = t % P.splits;
-  const int head = t / P.splits;
-  const int m0 = m_tile * 128;
-  const int kc0 = split * P.chunks_per_split;
-  const int kc1 = min(g.k_chunks, kc0 + P.chunks_per_split);
-  const int nk = kc1 - kc0;
-  const CUtensorMap *tm_a = P.a_map ? &tm_a1 : &tm_a0;
+  const int item0 = blockIdx.x * g.items_per_cta;
+  const int item1 = min(g.items, item0 + g.items_per_cta);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < g.stages; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->d_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->acc_full[i], 1);
+      mbar_init(&bars->acc_free[i], 4);
+    }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(tm_a);
+    prefetch_tmap(&tm_a0);
+    if (g.nprob > 1) prefetch_tmap(&tm_a1);
     prefetch_tmap(&tm_x);
   }
   if (warp == 1) {
@@ -103,50 +115,69 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int tx = kABytes + g.n_pad * 128;
-      int issued = 0;
-      for (int i = 0; i < nk; ++i, ++issued) {
-        const int st = i % g.stages;
-        if (i >= g.stages && !gwait(bars, g.err, &bars->empty[st], ((i / g.stages) - 1) & 1))
-          break;
-        uint8_t *a_dst = smem + st * stage_bytes;
-        uint8_t *x_dst = a_dst + kABytes;
-        const int k = (kc0 + i) * 64;
-        mbar_expect_tx(&bars->full[st], tx);
-        if (P.a_mn) {
-          // A[m][k] = A2d[head * K + k][m]: two 64-wide MN chunks, 64 K rows each
-          const int y = head * P.a_rows_per_head + k;
-          tma_load_2d(a_dst, tm_a, m0, y, &bars->full[st]);
-          tma_load_2d(a_dst + kABytes / 2, tm_a, m0 + 64, y, &bars->full[st]);
-        } else {
-          tma_load_2d(a_dst, tm_a, k, head * P.a_rows_per_head + m0, &bars->full[st]);
+      int c = 0;
+      bool ok = true;
+      for (int item = item0; ok && item < item1; ++item) {
+        const Item it = decode_item(g, item);
+        const GemmProblem &P = g.p[it.pi];
+        const CUtensorMap *tm_a = it.pi ? &tm_a1 : &tm_a0;
+        for (int i = 0; i < it.nk; ++i, ++c) {
+          const int st = c % g.stages;
+          if (c >= g.stages && !gwait(bars, g.err, &bars->empty[st], ((c / g.stages) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t *a_dst = smem + st * stage_bytes;
+          uint8_t *x_dst = a_dst + kABytes;
+          const int k = (it.kc0 + i) * 64;
+          mbar_expect_tx(&bars->full[st], tx);
+          if (P.a_mn) {
+            // A[m][k] = A2d[head * K + k][m]: two 64-wide MN chunks, 64 K rows each
+            const int y = it.head * P.a_rows_per_head + k;
+            tma_load_2d(a_dst, tm_a, it.m0, y, &bars->full[st]);
+            tma_load_2d(a_dst + kABytes / 2, tm_a, it.m0 + 64, y, &bars->full[st]);
+          } else {
+            tma_load_2d(a_dst, tm_a, k, it.head * P.a_rows_per_head + it.m0, &bars->full[st]);
+          }
+          tma_load_2d(x_dst, &tm_x, it.head * g.x_cols_per_head + k, 0, &bars->full[st]);
         }
-        tma_load_2d(x_dst, &tm_x, head * g.x_cols_per_head + k, 0, &bars->full[st]);
       }
-      for (int i = issued - g.stages; i < issued; ++i)
+      for (int i = c - g.stages; i < c; ++i)
         if (i >= 0) gwait(bars, g.err, &bars->full[i % g.stages], (i / g.stages) & 1);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, g.n_pad, P.a_mn, 0);
+      int c = 0;
       bool ok = true;
-      for (int i = 0; i < nk; ++i) {
-        const int st = i % g.stages;
-        if (!gwait(bars, g.err, &bars->full[st], (i / g.stages) & 1)) { ok = false; break; }
+      for (int item = item0, li = 0; ok && item < item1; ++item, ++li) {
+        const Item it = decode_item(g, item);
+        const GemmProblem &P = g.p[it.pi];
+        const uint32_t idesc = idesc_bf16(128, g.n_pad, P.a_mn, 0);
+        const int buf = li & 1;
+        const uint32_t acc = tmem + buf * g.n_pad;
+        if (li >= 2 && !gwait(bars, g.err, &bars->acc_free[buf], ((li >> 1) - 1) & 1)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + st * stage_bytes);
-        const uint32_t x_base = a_base + kABytes;
+        for (int i = 0; i < it.nk; ++i, ++c) {
+          const int st = c % g.stages;
+          if (!gwait(bars, g.err, &bars->full[st], (c / g.stages) & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + st * stage_bytes);
+          const uint32_t x_base = a_base + kABytes;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = P.a_mn ? sdesc(a_base + 2048 * k, kABytes / 2, 1024, 2)
-                                     : sdesc(a_base + 32 * k, 16, 1024, 2);
-          const uint64_t bd = sdesc(x_base + 32 * k, 16, 1024, 2);
-          umma_bf16(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = P.a_mn ? sdesc(a_base + 2048 * k, kABytes / 2, 1024, 2)
+                                       : sdesc(a_base + 32 * k, 16, 1024, 2);
+            const uint64_t bd = sdesc(x_base + 32 * k, 16, 1024, 2);
+            umma_bf16(acc, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&bars->empty[st]);
         }
-        umma_commit(&bars->empty[st]);
+        if (ok) umma_commit(&bars->acc_full[buf]);
       }
-      if (ok) umma_commit(&bars->d_full);
       umma_commit(&bars->drain);
       gwait(bars, g.err, &bars->drain, 0);
     }
@@ -154,10 +185,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     // epilogue: warps 2..5 cover TMEM lanes 64..127, 0..63 (lane quadrant = warp % 4)
     const int quad = warp & 3;
     const int ml = quad * 32 + lane;
-    const int m = m0 + ml;
-    if (nk > 0 && gwait(bars, g.err, &bars->d_full, 0)) {
+    for (int item = item0, li = 0; item < item1; ++item, ++li) {
+      const Item it = decode_item(g, item);
+      const GemmProblem &P = g.p[it.pi];
+      const int buf = li & 1;
+      if (!gwait(bars, g.err, &bars->acc_full[buf], (li >> 1) & 1)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+      const uint32_t taddr = tmem + buf * g.n_pad + (static_cast<uint32_t>(quad * 32) << 16);
+      const int m = it.m0 + ml;
       for (int c = 0; c < g.n_pad; c += 32) {
         uint32_t r[32];
         tmem_ld32(taddr + c, r);
@@ -169,10 +204,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (n < g.n) {
               const float v = __uint_as_float(r[j]);
               if (P.out_mode == kOutPartial) {
-                P.part[((long)split * g.n_total + g.n0 + n) * P.part_ld + P.part_col +
-                       (long)head * P.M + m] = v;
+                P.part[((long)it.split * g.n_total + g.n0 + n) * P.part_ld + P.part_col +
+                       (long)it.head * P.M + m] = v;
               } else {
-                const long idx = (long)n * P.ldy + (long)head * P.y_head + m;
+                const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
                 if (P.out_mode == kOutBf16)
                   static_cast<__nv_bfloat16 *>(P.out)[idx] = __float2bfloat16_rn(v);
                 else
@@ -183,6 +218,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_free[buf]);
     }
   }
   __syncthreads();
@@ -286,13 +323,13 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     g.x_cols_per_head = x_cols_per_head;
     g.err = err;
     g.tmem_cols = 32;
-    while (g.tmem_cols < g.n_pad) g.tmem_cols *= 2;
+    while (g.tmem_cols < 2 * g.n_pad) g.tmem_cols *= 2;
     const int stage_bytes = kABytes + g.n_pad * 128;
     // two CTAs per SM: half of the 227 KB of shared memory each
     g.stages = (232448 / 2 - 1024 - 256) / stage_bytes;
     if (g.stages > kMaxGemmStages) g.stages = kMaxGemmStages;
     CUtensorMap tm[2], tx;
-    int tiles = 0;
+    int items = 0;
     g.nprob = nops;
     for (int i = 0; i < nops; ++i) {
       const GemmOp &o = ops[i];
@@ -304,8 +341,8 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
       P.a_rows_per_head = o.a_mn ? K : o.M;
       P.splits = o.part ? o.splits : 1;
       P.chunks_per_split = (g.k_chunks + P.splits - 1) / P.splits;
-      P.tile_begin = tiles;
-      tiles += P.m_tiles * P.splits * o.heads;
+      P.item_begin = items;
+      items += P.m_tiles * P.splits * o.heads;
       P.out_mode = o.part ? kOutPartial : o.out_mode;
       P.out = o.out;
       P.ldy = o.ldy;
@@ -323,9 +360,13 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     }
     if (nops == 1) tm[1] = tm[0];
     if (!map2d(&tx, X + (long)n0 * x_cols, nn, x_cols, 64, g.n_pad)) return cudaErrorInvalidValue;
-    if (g.stages < 2) return cudaErrorInvalidValue;
+    // persistent CTAs: at most two per SM, each over a contiguous range of items
+    const int max_ctas = 2 * sm_count();
+    g.items = items;
+    g.items_per_cta = (items + max_ctas - 1) / max_ctas;
+    const int ctas = (items + g.items_per_cta - 1) / g.items_per_cta;
     const size_t smem = (size_t)g.stages * stage_bytes + 256 + 1024;
-    gemm_sm100_kernel<<<tiles, kThreads, smem, s>>>(tm[0], tm[1], tx, g);
+    gemm_sm100_kernel<<<ctas, kThreads, smem, s>>>(tm[0], tm[1], tx, g);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -27,9 +27,10 @@ struct GemmOp {
   int part_ld, part_col, splits;
 };
 
-// Kernel-side description of one problem of a launch.
+// Kernel-side description of one problem of a launch.  Its work items are
+// (head, split, m_tile) triples numbered from item_begin.
 struct GemmProblem {
-  int M, m_tiles, a_mn, a_map, a_rows_per_head, splits, chunks_per_split, tile_begin, out_mode;
+  int M, m_tiles, a_mn, a_map, a_rows_per_head, splits, chunks_per_split, item_begin, out_mode;
   void *out;
   long ldy, y_head;
   float *part;
@@ -39,6 +40,7 @@ struct GemmProblem {
 struct GemmLaunch {
   GemmProblem p[2];
   int nprob, n, n0, n_total, n_pad, k_chunks, x_cols_per_head, stages, tmem_cols;
+  int items, items_per_cta;
   int *err;
 };
 

@@ -24,11 +24,13 @@ struct GemvArgs {
 template <class TW, class TX, class TY>
 cudaError_t launch_gemv(const GemvArgs &a, int heads, cudaStream_t s);
 
+// xkv: `splits` partial sums [splits][batch][d_c + d_rope] of [W_DKV h ; W_KR h].
 template <class T>
-cudaError_t launch_append_finish(const float *xkv, int batch, int d_c, const RopeParams &rp,
-                                 const T *gamma, float eps, const int32_t *positions, T *pool,
-                                 int num_pages, int page_size, const int32_t *block_table,
-                                 int max_pages, int *err, cudaStream_t s);
+cudaError_t launch_append_finish(const float *xkv, int splits, int batch, int d_c,
+                                 const RopeParams &rp, const T *gamma, float eps,
+                                 const int32_t *positions, T *pool, int num_pages, int page_size,
+                                 const int32_t *block_table, int max_pages, int *err,
+                                 cudaStream_t s);
 
 template <class T>
 cudaError_t launch_rope_q(const float *qr, int batch, int n_heads, int d_c, const RopeParams &rp,

@@ -97,13 +97,20 @@ MLA_INST_GEMV(float, float, float)
 // ---------------------------------------------------------------------------
 
 template <class T>
-__global__ void append_finish(const float *xkv, int d_c, RopeParams rp, const T *gamma,
-                              float eps, const int32_t *positions, T *pool, int num_pages,
-                              int page_size, const int32_t *block_table, int max_pages,
-                              int *err) {
+__global__ void append_finish(const float *xkv, int splits, int batch, int d_c, RopeParams rp,
+                              const T *gamma, float eps, const int32_t *positions, T *pool,
+                              int num_pages, int page_size, const int32_t *block_table,
+                              int max_pages, int *err) {
+  // xkv holds `splits` partial sums [splits][batch][row] of [W_DKV h ; W_KR h]
+  extern __shared__ float x[];   // [row]
   const int b = blockIdx.x;
   const int row = d_c + rp.d_rope;
-  const float *x = xkv + (long)b * row;
+  for (int i = threadIdx.x; i < row; i += blockDim.x) {
+    float v = 0.f;
+    for (int sp = 0; sp < splits; ++sp) v += xkv[((long)sp * batch + b) * row + i];
+    x[i] = v;
+  }
+  __syncthreads();
   __shared__ float red[32];
   __shared__ float inv_rms;
   float ss = 0.f;
@@ -139,21 +146,24 @@ __global__ void append_finish(const float *xkv, int d_c, RopeParams rp, const T 
 }
 
 template <class T>
-cudaError_t launch_append_finish(const float *xkv, int batch, int d_c, const RopeParams &rp,
-                                 const T *gamma, float eps, const int32_t *positions, T *pool,
-                                 int num_pages, int page_size, const int32_t *block_table,
-                                 int max_pages, int *err, cudaStream_t s) {
-  append_finish<T><<<batch, 256, 0, s>>>(xkv, d_c, rp, gamma, eps, positions, pool, num_pages,
-                                          page_size, block_table, max_pages, err);
+cudaError_t launch_append_finish(const float *xkv, int splits, int batch, int d_c,
+                                 const RopeParams &rp, const T *gamma, float eps,
+                                 const int32_t *positions, T *pool, int num_pages, int page_size,
+                                 const int32_t *block_table, int max_pages, int *err,
+                                 cudaStream_t s) {
+  const size_t smem = (d_c + rp.d_rope) * sizeof(float);
+  append_finish<T><<<batch, 256, smem, s>>>(xkv, splits, batch, d_c, rp, gamma, eps, positions,
+                                            pool, num_pages, page_size, block_table, max_pages,
+                                            err);
   return cudaGetLastError();
 }
-template cudaError_t launch_append_finish<float>(const float *, int, int, const RopeParams &,
+template cudaError_t launch_append_finish<float>(const float *, int, int, int, const RopeParams &,
                                                  const float *, float, const int32_t *, float *,
                                                  int, int, const int32_t *, int, int *,
                                                  cudaStream_t);
 template cudaError_t launch_append_finish<__nv_bfloat16>(
-    const float *, int, int, const RopeParams &, const __nv_bfloat16 *, float, const int32_t *,
-    __nv_bfloat16 *, int, int, const int32_t *, int, int *, cudaStream_t);
+    const float *, int, int, int, const RopeParams &, const __nv_bfloat16 *, float,
+    const int32_t *, __nv_bfloat16 *, int, int, const int32_t *, int, int *, cudaStream_t);
 
 // ---------------------------------------------------------------------------
 // q_R = RoPE_pos(W_QR c_Q) written into the tail of each q_lat row
@@ -162,19 +172,27 @@ template cudaError_t launch_append_finish<__nv_bfloat16>(
 template <class T>
 __global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
                        const int32_t *positions, T *q_lat) {
+  // the rotation angles pos * theta_i are the same for every head of a sequence
+  __shared__ float cs[64], sn[64];
   const int b = blockIdx.x;
   const int half = rp.d_rope / 2;
   const int pos = positions[b];
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    double s, c;
+    sincos((double)pos * rp.theta[i], &s, &c);
+    cs[i] = (float)c;
+    sn[i] = (float)s;
+  }
+  __syncthreads();
   for (int t = threadIdx.x; t < n_heads * half; t += blockDim.x) {
     const int h = t / half, i = t % half;
     int j0, j1;
     rope_idx(rp, i, j0, j1);
     const float *src = qr + ((long)b * n_heads + h) * rp.d_rope;
-    float x0 = src[j0], x1 = src[j1];
-    rope_pair(rp, i, pos, x0, x1);
+    const float x0 = src[j0], x1 = src[j1];
     T *dst = q_lat + ((long)b * n_heads + h) * (d_c + rp.d_rope) + d_c;
-    dst[j0] = st_cast<T>(x0);
-    dst[j1] = st_cast<T>(x1);
+    dst[j0] = st_cast<T>(x0 * cs[i] - x1 * sn[i]);
+    dst[j1] = st_cast<T>(x0 * sn[i] + x1 * cs[i]);
   }
 }
 
@@ -430,15 +448,38 @@ template cudaError_t launch_attn_simt<float>(const AttnArgs &, int, cudaStream_t
 // z = sum_j w_j O_j / sum_j w_j l_j with w_j = exp(m_j - max_j m_j), and
 // lse = max_j m_j + log(sum_j w_j l_j): the standard merge of partial softmaxes.
 
+constexpr int kCombineHeads = 16;     // heads per block
+constexpr int kCombineMaxPieces = 64; // pieces whose weights are staged in shared memory
+
+template <class T> struct Vec4Out;
+template <> struct Vec4Out<float> {
+  static __device__ __forceinline__ void store(float *p, float4 v) {
+    *reinterpret_cast<float4 *>(p) = v;
+  }
+};
+template <> struct Vec4Out<__nv_bfloat16> {
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = u;
+  }
+};
+
 template <class T>
 __global__ void combine_kernel(AttnArgs a) {
   const int b = blockIdx.x;
+  const int h0 = blockIdx.y * kCombineHeads;
   const PlanHeader hdr = *a.hdr;
   T *zb = reinterpret_cast<T *>(a.z) + (long)b * a.n_heads * a.d_c;
   if (a.bad[b]) {
-    for (int i = threadIdx.x; i < a.n_heads * a.d_c; i += blockDim.x) zb[i] = st_cast<T>(0.f);
+    for (int i = threadIdx.x; i < kCombineHeads * a.d_c; i += blockDim.x) {
+      const int h = h0 + i / a.d_c;
+      if (h < a.n_heads) zb[(long)h * a.d_c + i % a.d_c] = st_cast<T>(0.f);
+    }
     if (a.lse)
-      for (int h = threadIdx.x; h < a.n_heads; h += blockDim.x)
+      for (int h = h0 + threadIdx.x; h < min(a.n_heads, h0 + kCombineHeads); h += blockDim.x)
         a.lse[(long)b * a.n_heads + h] = -INFINITY;
     return;
   }
@@ -446,7 +487,11 @@ __global__ void combine_kernel(AttnArgs a) {
   if (pb < 0) return;
   const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
   const int pieces = (s1 - 1) / hdr.quota - s0 / hdr.quota + 1;
-  for (int h = blockIdx.y; h < a.n_heads; h += gridDim.y) {
+  __shared__ float wgt[kCombineMaxPieces][kCombineHeads];
+  // per head: w_j = exp(m_j - M) / sum_j exp(m_j - M) l_j, lse = M + log(sum)
+  for (int hh = threadIdx.x; hh < kCombineHeads; hh += blockDim.x) {
+    const int h = h0 + hh;
+    if (h >= a.n_heads) continue;
     float M = -INFINITY;
     for (int j = 0; j < pieces; ++j) M = fmaxf(M, a.part_m[(long)(pb + j) * a.n_heads + h]);
     float den = 0.f;
@@ -455,22 +500,45 @@ __global__ void combine_kernel(AttnArgs a) {
       den += expf(a.part_m[idx] - M) * a.part_l[idx];
     }
     const float inv = 1.f / den;
-    for (int d = threadIdx.x; d < a.d_c; d += blockDim.x) {
-      float v = 0.f;
-      for (int j = 0; j < pieces; ++j) {
-        const long idx = (long)(pb + j) * a.n_heads + h;
-        v += expf(a.part_m[idx] - M) * a.part_O[idx * a.d_c + d];
+    for (int j = 0; j < pieces && j < kCombineMaxPieces; ++j)
+      wgt[j][hh] = expf(a.part_m[(long)(pb + j) * a.n_heads + h] - M) * inv;
+    if (a.lse) a.lse[(long)b * a.n_heads + h] = M + logf(den);
+  }
+  __syncthreads();
+  const int nvec = a.d_c / 4;
+  for (int i = threadIdx.x; i < kCombineHeads * nvec; i += blockDim.x) {
+    const int hh = i / nvec, d = (i % nvec) * 4;
+    const int h = h0 + hh;
+    if (h >= a.n_heads) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < pieces; ++j) {
+      const long idx = (long)(pb + j) * a.n_heads + h;
+      float w;
+      if (j < kCombineMaxPieces) {
+        w = wgt[j][hh];
+      } else {  // very long splits: recompute the weight (rare)
+        float M = -INFINITY, den = 0.f;
+        for (int q = 0; q < pieces; ++q) M = fmaxf(M, a.part_m[(long)(pb + q) * a.n_heads + h]);
+        for (int q = 0; q < pieces; ++q) {
+          const long iq = (long)(pb + q) * a.n_heads + h;
+          den += expf(a.part_m[iq] - M) * a.part_l[iq];
+        }
+        w = expf(a.part_m[idx] - M) / den;
       }
-      zb[(long)h * a.d_c + d] = st_cast<T>(v * inv);
+      const float4 v = *reinterpret_cast<const float4 *>(a.part_O + idx * a.d_c + d);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
     }
-    if (a.lse && threadIdx.x == 0) a.lse[(long)b * a.n_heads + h] = M + logf(den);
+    Vec4Out<T>::store(zb + (long)h * a.d_c + d, acc);
   }
 }
 
 template <class T>
 cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s) {
-  dim3 grid(a.batch, a.n_heads < 16 ? a.n_heads : 16);
-  combine_kernel<T><<<grid, 128, 0, s>>>(a);
+  dim3 grid(a.batch, (a.n_heads + kCombineHeads - 1) / kCombineHeads);
+  combine_kernel<T><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 template cudaError_t launch_combine<float>(const AttnArgs &, cudaStream_t);

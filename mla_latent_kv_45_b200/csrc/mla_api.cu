@@ -82,7 +82,7 @@ mla_status check_dims(const mla_dims *d) {
   if (!(d->rope_base > 0.0) || !(d->rms_eps >= 0.0) || !(d->softmax_scale >= 0.0))
     return MLA_ERR_INVALID_ARG;
   if (d->dtype == MLA_FP32) {
-    if (d->n_heads > 256 || d->d_c > 1024 || d->d_nope > 256 || d->d_v > 256)
+    if (d->n_heads > 256 || d->d_c > 1024 || (d->d_c % 4) || d->d_nope > 256 || d->d_v > 256)
       return MLA_ERR_UNSUPPORTED;
   } else {
     if (d->n_heads != 128 || d->d_c != 512 || d->d_rope != 64 || d->d_nope != 128 ||
@@ -180,15 +180,17 @@ mla_status mla_cache_append(const mla_dims *dims, const mla_paged_cache *cache, 
     MLA_TRY((gemv<float, float, float>(W_KR, 0, d_model, 1, h, 0, d_model, xkv + d.d_c, 0, row,
                                        d.d_rope, d_model, batch, 1, s)));
     return cuda_ok(launch_append_finish<float>(
-        xkv, batch, d.d_c, rp, static_cast<const float *>(gamma), (float)d.rms_eps, positions,
+        xkv, 1, batch, d.d_c, rp, static_cast<const float *>(gamma), (float)d.rms_eps, positions,
         static_cast<float *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
         cache->max_pages_per_seq, err, s));
   }
+  const float *parts = nullptr;
+  int splits = 1;
   MLA_TRY(cuda_ok(sm100::append_proj(static_cast<const bf16 *>(h), static_cast<const bf16 *>(W_DKV),
                                      static_cast<const bf16 *>(W_KR), batch, d_model, xkv,
-                                     at(ws, L.gemm), err, s)));
+                                     at(ws, L.gemm), err, &parts, &splits, s)));
   return cuda_ok(launch_append_finish<bf16>(
-      xkv, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
+      parts, splits, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
       static_cast<bf16 *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
       cache->max_pages_per_seq, err, s));
 }

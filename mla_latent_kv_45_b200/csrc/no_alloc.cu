@@ -96,7 +96,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
       (d.rope_layout != MLA_ROPE_INTERLEAVED && d.rope_layout != MLA_ROPE_HALF))
     return MLA_ERR_INVALID_ARG;
   if (d.dtype == MLA_FP32 &&
-      (d.n_heads > 256 || d.d_c > 1024 || d.d_nope > 256 || d.d_v > 256))
+      (d.n_heads > 256 || d.d_c > 1024 || (d.d_c % 4) || d.d_nope > 256 || d.d_v > 256))
     return MLA_ERR_UNSUPPORTED;
   if (d.dtype == MLA_BF16 && (d.n_heads != 128 || d.d_c != 512 || d.d_rope != 64 ||
                               d.d_nope != 128 || d.d_v != 128 || d.page_size != 64))

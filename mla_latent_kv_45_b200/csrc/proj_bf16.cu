@@ -66,19 +66,23 @@ size_t gemm_workspace_bytes(int batch, int d_model, int d_q, int n_heads, const 
 }
 
 cudaError_t append_proj(const bf16 *h, const bf16 *W_DKV, const bf16 *W_KR, int batch,
-                        int d_model, float *xkv, void *gemm_ws, int *err, cudaStream_t s) {
+                        int d_model, float *xkv, void *gemm_ws, int *err, const float **out,
+                        int *splits_out, cudaStream_t s) {
   const int splits = gemm_splits(5, 1, d_model / 64);
   GemmOp ops[2] = {op(W_DKV, 512, 1, 0), op(W_KR, 64, 1, 0)};
+  *splits_out = splits;
   if (splits == 1) {
     direct(ops[0], kOutF32, xkv, 576);
     direct(ops[1], kOutF32, xkv + 512, 576);
+    *out = xkv;
     return gemm(ops, 2, h, batch, d_model, d_model, 0, err, s);
   }
+  // the partial sums are added by the append epilogue kernel
   float *part = static_cast<float *>(gemm_ws);
   partial(ops[0], part, 576, 0, splits);
   partial(ops[1], part, 576, 512, splits);
-  TRY(gemm(ops, 2, h, batch, d_model, d_model, 0, err, s));
-  return gemm_reduce(part, splits, batch, 576, 576, xkv, 576, false, s);
+  *out = part;
+  return gemm(ops, 2, h, batch, d_model, d_model, 0, err, s);
 }
 
 cudaError_t absorb_proj(const bf16 *x, const bf16 *W_DQ, const bf16 *W_UQ, const bf16 *W_QR,

@@ -19,10 +19,12 @@ constexpr int kAttnMinPages = 4;
 // Workspace bytes the projections need beyond the fp32 intermediates.
 size_t gemm_workspace_bytes(int batch, int d_model, int d_q, int n_heads, const mla_dims &d);
 
-// xkv[b] = [W_DKV h_b ; W_KR h_b] in fp32 ([batch][576]).
+// [W_DKV h_b ; W_KR h_b] in fp32 as `*splits` partial sums [splits][batch][576]
+// at *out (xkv itself when there is one split, else the GEMM workspace).
 cudaError_t append_proj(const __nv_bfloat16 *h, const __nv_bfloat16 *W_DKV,
                         const __nv_bfloat16 *W_KR, int batch, int d_model, float *xkv,
-                        void *gemm_ws, int *err, cudaStream_t s);
+                        void *gemm_ws, int *err, const float **out, int *splits,
+                        cudaStream_t s);
 
 // c_Q (bf16, when W_DQ), q_C (bf16), raw q_R (fp32, not yet rotated) and the
 // absorbed content half q_lat[b][i][0:512] = W_UK,i^T q_C,i (bf16).

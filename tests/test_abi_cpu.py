@@ -61,6 +61,7 @@ def test_workspace_size(lib):
     assert L.mla_workspace_size(V2, 64, 5120, 1536, 8) < n
     assert L.mla_workspace_size(L.Dims(128, 513, 64, 128, 128, 64), 4, 5120, 0, 0) == 0
     assert L.mla_workspace_size(TINY, 2, 64, 0, 0) > 0
+    assert L.mla_workspace_size(L.Dims(4, 18, 8, 8, 8, 16, L.MLA_FP32), 2, 64, 0, 0) == 0
 
 
 def test_decode_attn_host_checks(lib):
