@@ -357,8 +357,9 @@ def run_mine(args):
 
 
 # Launches of this library per decode step (checked against the ncu launch list):
-# append 3 (2 projections + finish), absorb_q 5 (W_DQ, W_UQ, W_QR, W_UK, RoPE),
-# decode_attn 3 (plan, attention, merge), unabsorb_out 2 (W_UV, W_O).
+# append 2 (W_DKV+W_KR projection, RMSNorm/RoPE/page write), absorb_q 5 (W_DQ,
+# its split-K reduce, W_UQ+W_QR, W_UK, RoPE), decode_attn 3 (plan, attention,
+# merge), unabsorb_out 3 (W_UV, W_O, its split-K reduce).
 LAUNCHES_PER_STEP = 13
 
 

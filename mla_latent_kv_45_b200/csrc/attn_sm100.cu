@@ -14,8 +14,9 @@
 //  * Rows of each 64-row page are split between the pair: CTA r scores its
 //    own 32 rows [32 r, 32 r + 32) over all 576 columns (tcgen05.mma,
 //    M = 128 heads, N = 32 rows, K = 576), so no partial score is exchanged.
-//    q_lat is the A operand: 448 of its columns sit in TMEM, the last 128
-//    (latent 448..511 and k_R) in shared memory.
+//    q_lat is the A operand: 384 of its columns sit in TMEM, the last 192
+//    (latent 384..511 and k_R) in shared memory.  S has two TMEM buffers, so
+//    the scores of the next tile are computed while this tile's are read.
 //  * Each CTA turns its own rows into P (bf16, exp2 domain) relative to a
 //    reference max that both CTAs share, and sends its P half plus the
 //    reference it used to the partner with st.async stores (8.5 KB per tile,
@@ -26,7 +27,10 @@
 //  * O_half += P . V_half on tcgen05 (A = the 64-row P tile in shared
 //    memory, B = the page's latent half: the CTA's own rows come with its
 //    full-width tile, the partner's 32 rows are loaded separately and are
-//    normally L2 hits because the partner streams the same page).
+//    normally L2 hits because the partner streams the same page).  The P tile
+//    is written over the stage's own rows' other latent half, which only S
+//    reads: once both CTAs' S of the tile is complete they say so to each
+//    other and write their P halves there.
 //  * Row sums are taken from the bf16 P both CTAs feed the MMA (own and
 //    received halves), so no sum is exchanged; the epilogue divides O_half.
 //  * Two softmax warpgroups (TMEM lane = head): warpgroup g owns 16 of the
@@ -60,17 +64,20 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 96;   // + producer, score issuer, P.V issuer
 constexpr int kWarpProd = 8, kWarpS = 9, kWarpPV = 10;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kSleepNs = 20000;   // suspend hint of a waiting thread (woken at completion)
 
 // Shared memory (byte offsets from a 1024-byte aligned base).
 constexpr int kChunk = kOwn * 128;               // 32 rows x 64 bf16, 128-byte swizzle
 constexpr int kQChunk = kHeads * 128;            // 128 heads x 64 bf16
-constexpr int kOffQ = 0;                         // q_lat columns 448..575 (2 chunks)
-constexpr int kOffStage = kOffQ + 2 * kQChunk;
+constexpr int kQSmem = 3;                        // q_lat columns 384..575 in shared memory
+constexpr int kOffQ = 0;
+constexpr int kOffStage = kOffQ + kQSmem * kQChunk;
 constexpr int kRegionB = 9 * kChunk;             // own rows: 9 chunks x 64 columns
 constexpr int kStageBytes = kRegionB + 4 * kChunk;  // + partner rows, own latent half
-constexpr int kPBytes = kHeads * 128;            // P tile: 128 heads x 64 rows bf16
-constexpr int kOffP = kOffStage + kStages * kStageBytes;   // two P tiles
-constexpr int kOffRef = kOffP + 2 * kPBytes;     // two x 128 received reference maxima
+// The P tile of a tile (128 heads x 64 rows bf16, 16 KB) is written into its
+// stage's own rows' other latent half (chunks 4(1-r)..4(1-r)+3): S is the only
+// reader of those chunks, so they are dead once S of the tile is complete.
+constexpr int kOffRef = kOffStage + kStages * kStageBytes;  // two x 128 received reference maxima
 constexpr int kOffRed = kOffRef + 1024;          // 2 x 128 floats: per-warpgroup scratch
 constexpr int kOffBar = kOffRed + 1024;
 constexpr int kSmemBytes = kOffBar + 512 + 1024;
@@ -78,8 +85,9 @@ constexpr uint32_t kMsgBytes = kHeads * kOwn * 2 + kHeads * 4;   // P half + ref
 
 // TMEM columns
 constexpr uint32_t kTmemO = 0;     // O_half: 256 fp32 columns
-constexpr uint32_t kTmemQ = 256;   // q_lat columns 0..447: 224 columns of bf16 pairs
-constexpr uint32_t kTmemS = 480;   // S: 32 fp32 columns
+constexpr uint32_t kTmemQ = 256;   // q_lat columns 0..383: 192 columns of bf16 pairs
+constexpr uint32_t kTmemS = 448;   // S: two buffers of 32 fp32 columns
+constexpr int kQTmemDims = 384;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescS = idesc_bf16(128, kOwn, 0, 0);  // A = q_lat, B = own rows (K-major)
@@ -87,11 +95,12 @@ constexpr uint32_t kIdescPV = idesc_bf16(128, 256, 0, 1);  // A = P (K-major), B
 
 struct Bars {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_tmem, q_smem, q_free, s_full, s_free, drain_s, drain_pv;
+  uint64_t q_tmem, q_smem, q_free, drain_s, drain_pv;
+  uint64_t s_full[2], s_free[2];  // score buffer i written / read
   uint64_t pv_done[2];     // P.V of the tile using P tile slot i completed
   uint64_t p_ready[2];     // own P half written and partner half final (8 softmax warps)
   uint64_t p_rx[2];        // partner's P half + references landed (tx count)
-  uint64_t p_slot_free[2]; // partner's P tile slot may be overwritten (remote arrive)
+  uint64_t p_slot_free[2]; // partner's S of the tile done: its P tile may be written (remote arrive)
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -108,7 +117,9 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, uint64_t *bar, uint32_t p
   if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
+    if (kCluster ? mbar_try_wait_cluster_sleep(a, parity, kSleepNs)
+                 : mbar_try_wait_sleep(a, parity, kSleepNs))
+      return true;
     if (c.bars->abort) return false;
     if (globaltimer() - t0 > kTimeoutNs) {
       set_error(c.err, kErrTimeout);
@@ -173,12 +184,12 @@ struct TileCursor {
   __device__ __forceinline__ bool last() const { return lp == seg.lp1 - 1; }
 };
 
-// Stages q_lat[b][h][0:448] into TMEM lane h (224 columns of bf16 pairs);
-// warpgroup 0 writes columns [0, 128), warpgroup 1 columns [128, 224).
+// Stages q_lat[b][h][0:384] into TMEM lane h (192 columns of bf16 pairs);
+// warpgroup 0 writes columns [0, 96), warpgroup 1 columns [96, 192).
 __device__ __forceinline__ void stage_q(const AttnArgs &a, int b, int h, int g, uint32_t taddr) {
   const uint4 *src = reinterpret_cast<const uint4 *>(
       reinterpret_cast<const __nv_bfloat16 *>(a.q_lat) + ((long)b * kHeads + h) * kRow);
-  const int b0 = g ? 4 : 0, b1 = g ? 7 : 4;       // blocks of 32 TMEM columns
+  const int b0 = g ? 3 : 0, b1 = g ? 6 : 3;       // blocks of 32 TMEM columns
   for (int bb = b0; bb < b1; ++bb) {
     uint32_t v[32];
 #pragma unroll
@@ -214,8 +225,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&bars->q_tmem, 8);
     mbar_init(&bars->q_smem, 1);
     mbar_init(&bars->q_free, 1);
-    mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->s_free[i], 8);
+    }
     mbar_init(&bars->drain_s, 1);
     mbar_init(&bars->drain_pv, 1);
     for (int i = 0; i < 2; ++i) {
@@ -278,6 +291,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ---------------------------------------- score MMA issuer (+ q_lat smem part)
     if (lane == 0) {
       const uint32_t q_base = smem_u32(smem + kOffQ);
+      const uint64_t qd = sdesc(q_base, 16, 1024, 2);
       int tile = 0;
       bool ok = true;
       for (; cur.valid; cur.advance(a), ++tile) {
@@ -285,26 +299,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (cur.first()) {
           // the previous segment's score MMAs must finish before q_lat is replaced
           if (cur.nseg > 0 && !wait_bar<false>(ctx, &bars->q_free, (cur.nseg - 1) & 1)) { ok = false; break; }
-          mbar_expect_tx(&bars->q_smem, 2 * kQChunk);
-          tma_load_2d(smem + kOffQ, &tm_q, 448, cur.seg.b * kHeads, &bars->q_smem);
-          tma_load_2d(smem + kOffQ + kQChunk, &tm_q, 512, cur.seg.b * kHeads, &bars->q_smem);
+          mbar_expect_tx(&bars->q_smem, kQSmem * kQChunk);
+          for (int c = 0; c < kQSmem; ++c)
+            tma_load_2d(smem + kOffQ + c * kQChunk, &tm_q, kQTmemDims + 64 * c, cur.seg.b * kHeads,
+                        &bars->q_smem);
           if (!wait_bar<false>(ctx, &bars->q_smem, cur.nseg & 1)) { ok = false; break; }
           if (!wait_bar<false>(ctx, &bars->q_tmem, cur.nseg & 1)) { ok = false; break; }
         }
         if (!wait_bar<false>(ctx, &bars->full[st], (tile / kStages) & 1)) { ok = false; break; }
-        if (tile > 0 && !wait_bar<false>(ctx, &bars->s_free, (tile - 1) & 1)) { ok = false; break; }
+        // score buffer tile&1 was last used by tile-2
+        const int sb = tile & 1;
+        if (tile >= 2 && !wait_bar<false>(ctx, &bars->s_free[sb], ((tile >> 1) - 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + kOffStage + st * kStageBytes);
-        for (int s = 0; s < 28; ++s)        // q_lat columns 0..447 from TMEM
-          umma_bf16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * s,
-                       sdesc(k_base + (s >> 2) * kChunk + 32 * (s & 3), 16, 1024, 2), kIdescS,
+        // descriptors advance by address >> 4 in their low field (no carry: < 256 KB)
+        const uint64_t kd = sdesc(smem_u32(smem + kOffStage + st * kStageBytes), 16, 1024, 2);
+        const uint32_t sd = tmem + kTmemS + 32 * sb;
+#pragma unroll
+        for (int s = 0; s < kQTmemDims / 16; ++s)   // q_lat columns 0..383 from TMEM
+          umma_bf16_ts(sd, tmem + kTmemQ + 8 * s,
+                       kd + (uint64_t)(((s >> 2) * kChunk + 32 * (s & 3)) >> 4), kIdescS,
                        s ? 1u : 0u);
-        for (int s = 0; s < 8; ++s)         // columns 448..575 from shared memory
-          umma_bf16(tmem + kTmemS, sdesc(q_base + (s >> 2) * kQChunk + 32 * (s & 3), 16, 1024, 2),
-                    sdesc(k_base + (7 + (s >> 2)) * kChunk + 32 * (s & 3), 16, 1024, 2), kIdescS,
-                    1u);
+#pragma unroll
+        for (int s = 0; s < 4 * kQSmem; ++s)         // columns 384..575 from shared memory
+          umma_bf16(sd, qd + (uint64_t)(((s >> 2) * kQChunk + 32 * (s & 3)) >> 4),
+                    kd + (uint64_t)(((kQTmemDims / 64 + (s >> 2)) * kChunk + 32 * (s & 3)) >> 4),
+                    kIdescS, 1u);
         if (cur.last()) umma_commit(&bars->q_free);
-        umma_commit(&bars->s_full);
+        umma_commit(&bars->s_full[sb]);
       }
       (void)ok;
       umma_commit(&bars->drain_s);
@@ -313,7 +334,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpPV) {
     // ------------------------------------------------------------ P.V MMA issuer
     if (lane == 0) {
-      const uint32_t p_base = smem_u32(smem + kOffP);
       int tile = 0;
       for (; cur.valid; cur.advance(a), ++tile) {
         const int st = tile % kStages;
@@ -321,13 +341,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!wait_bar<false>(ctx, &bars->p_ready[pb], (tile >> 1) & 1)) break;
         tc_fence_after();
         const uint32_t v_base = smem_u32(smem + kOffStage + st * kStageBytes);
+        const uint32_t p_base = v_base + 4 * (1 - rank) * kChunk;
         const bool first = cur.first();
         for (int k = 0; k < kPage / 16; ++k) {
           // rows [16 k, 16 k + 16) of the page: own rows (full-width tile, latent
           // half = chunks 4r..4r+3) or partner rows (region B); chunks 4 KB apart
           const bool own = (k >> 1) == (int)rank;
           const uint32_t vb = v_base + (own ? 4 * rank * kChunk : kRegionB) + (k & 1) * 2048;
-          umma_bf16(tmem + kTmemO, sdesc(p_base + pb * kPBytes + 32 * k, 16, 1024, 2),
+          umma_bf16(tmem + kTmemO, sdesc(p_base + 32 * k, 16, 1024, 2),
                     sdesc(vb, kChunk, 1024, 2), kIdescPV, (first && k == 0) ? 0u : 1u);
         }
         umma_commit(&bars->pv_done[pb]);
@@ -343,12 +364,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float *red = reinterpret_cast<float *>(smem + kOffRed);   // [2][128]
     const float *refs = reinterpret_cast<const float *>(smem + kOffRef);  // [2][128]
-    uint8_t *pt = smem + kOffP;
-    // P tile row h: 16-byte chunk c (rows 8c..8c+7 of the page) at h*128 + ((c ^ (h&7)) << 4)
+    // P tile row h: 16-byte chunk c (rows 8c..8c+7 of the page) at h*128 + ((c ^ (h&7)) << 4);
+    // the tile sits in chunks 4(1-r).. of the stage here and in chunks 4r.. at the partner
     const int c_own = 4 * rank + 2 * g;      // this thread's two own chunks: c_own, c_own + 1
     const int c_peer = 4 * (1 - rank) + 2 * g;  // and the matching partner chunks
-    const uint32_t p_local = smem_u32(pt) + h * 128;
-    const uint32_t p_remote = mapa(p_local, peer);
+    auto p_row = [&](int j) {
+      return smem + kOffStage + (j % kStages) * kStageBytes + 4 * (1 - rank) * kChunk + h * 128;
+    };
+    const uint32_t p_remote0 = mapa(smem_u32(smem + kOffStage + 4 * rank * kChunk) + h * 128, peer);
     const uint32_t ref_remote = mapa(smem_u32(smem + kOffRef) + h * 4, peer);
     const uint32_t rx_remote = mapa(smem_u32(&bars->p_rx[0]), peer);
     const uint32_t slot_free_remote = mapa(smem_u32(&bars->p_slot_free[0]), peer);
@@ -367,14 +390,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&bars->q_tmem);
         m_run = -INFINITY;
       }
-      if (!wait_bar<false>(ctx, &bars->s_full, j & 1)) return false;
+      const int sb = j & 1;
+      if (!wait_bar<false>(ctx, &bars->s_full[sb], (j >> 1) & 1)) return false;
       tc_fence_after();
       float sv[16];
-      tmem_ld16f(tmem + lane_off + kTmemS + 16 * g, sv);
+      tmem_ld16f(tmem + lane_off + kTmemS + 32 * sb + 16 * g, sv);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_free);
+      if (lane == 0) mbar_arrive(&bars->s_free[sb]);
       const int rows_valid = tc.seg.len - tc.lp * kPage;          // >= 1
       const int own_valid = min(max(rows_valid - kOwn * (int)rank, 0), kOwn);
       const int mine = own_valid - 16 * g;                          // valid among my 16
@@ -412,21 +436,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       const int pb = j & 1;
-      if (j >= 2) {
-        // this CTA's P.V of tile j-2 read P tile pb: free it locally and for the partner
-        if (!wait_bar<false>(ctx, &bars->pv_done[pb], ((j >> 1) - 1) & 1)) return false;
-        if (threadIdx.x == 0) mbar_arrive_cluster_relaxed(slot_free_remote + pb * 8);
-        if (!wait_bar<true>(ctx, &bars->p_slot_free[pb], ((j >> 1) - 1) & 1)) return false;
-      }
+      // S of tile j is complete here, so the dead chunks holding this CTA's P
+      // tile of tile j may be written; tell the partner, and wait for its word
+      if (threadIdx.x == 0) mbar_arrive_cluster_relaxed(slot_free_remote + pb * 8);
+      if (!wait_bar<true>(ctx, &bars->p_slot_free[pb], (j >> 1) & 1)) return false;
       const uint4 v0 = make_uint4(w[0], w[1], w[2], w[3]);
       const uint4 v1 = make_uint4(w[4], w[5], w[6], w[7]);
-      const uint32_t o0 = pb * kPBytes + ((c_own ^ (h & 7)) << 4);
-      const uint32_t o1 = pb * kPBytes + (((c_own + 1) ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4 *>(pt + h * 128 + o0) = v0;
-      *reinterpret_cast<uint4 *>(pt + h * 128 + o1) = v1;
+      const uint32_t o0 = (c_own ^ (h & 7)) << 4;
+      const uint32_t o1 = ((c_own + 1) ^ (h & 7)) << 4;
+      uint8_t *prow = p_row(j);
+      *reinterpret_cast<uint4 *>(prow + o0) = v0;
+      *reinterpret_cast<uint4 *>(prow + o1) = v1;
       const uint32_t mb = rx_remote + pb * 8;
-      st_async_v4u(p_remote + o0, v0, mb);
-      st_async_v4u(p_remote + o1, v1, mb);
+      const uint32_t rrow = p_remote0 + (j % kStages) * kStageBytes;
+      st_async_v4u(rrow + o0, v0, mb);
+      st_async_v4u(rrow + o1, v1, mb);
       if (g == 0) st_async_f32(ref_remote + pb * 512, ref_own, mb);
       return true;
     };
@@ -443,7 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float f_own = ref_own < m_new ? ex2(ref_own - m_new) : 1.f;
       const float f_peer = ref_p < m_new ? ex2(ref_p - m_new) : 1.f;
       const float alpha = (first || !(m_new > m_run)) ? 1.f : ex2(m_run - m_new);
-      uint8_t *row = pt + pb * kPBytes + h * 128;
+      uint8_t *row = p_row(j);
       uint4 *q0 = reinterpret_cast<uint4 *>(row + ((c_own ^ (h & 7)) << 4));
       uint4 *q1 = reinterpret_cast<uint4 *>(row + (((c_own + 1) ^ (h & 7)) << 4));
       uint4 *q2 = reinterpret_cast<uint4 *>(row + ((c_peer ^ (h & 7)) << 4));

@@ -47,7 +47,7 @@ __device__ __forceinline__ bool gwait(Bars *bars, int *err, uint64_t *bar, uint3
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait_sleep(a, parity, 20000)) return true;
     if (bars->abort) return false;
     if (globaltimer() - t0 > kTimeoutNs) {
       set_error(err, kErrTimeout);
