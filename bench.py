@@ -223,25 +223,16 @@ def run_mine(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st = L.mla_get_device_error(layer.ws)
+    st = layer.device_error()
     if st != 0:
         raise RuntimeError(f"device error {L.STATUS.get(st)} during warm-up")
 
-    # per-call events inside the timed region (same stream as the launches)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    w = layer.w
+    # per-call events inside the timed region: the append on the layer's side
+    # stream, the other calls on the main stream (see DecodeLayer.step)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
 
     def timed_step(e):
-        e[0].record(stream)
-        L.mla_cache_append(dims, cache, hd, w["W_DKV"], w["W_KR"], w["gamma"], pos, layer.ws)
-        e[1].record(stream)
-        L.mla_absorb_q(dims, hd, w["W_DQ"], w["W_UQ"], w["W_QR"], w["W_UK"], pos, layer.q_lat,
-                       layer.ws)
-        e[2].record(stream)
-        L.mla_decode_attn(dims, cache, layer.q_lat, layer.z, layer.lse, args.num_splits, layer.ws)
-        e[3].record(stream)
-        L.mla_unabsorb_out(dims, layer.z, w["W_UV"], w["W_O"], layer.out, layer.ws)
-        e[4].record(stream)
+        layer.step(cache, hd, pos, stream, e)
 
     gpu_id = torch.cuda.get_device_properties(dev).uuid
     gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else gpu_id
@@ -263,8 +254,9 @@ def run_mine(args):
     if world > 1:
         torch.distributed.barrier()
     elapsed = start.elapsed_time(end)  # ms
-    per_call = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in ev])
-    st = L.mla_get_device_error(layer.ws)
+    per_call = np.array([[e[0].elapsed_time(e[1]), e[2].elapsed_time(e[3]),
+                          e[4].elapsed_time(e[5]), e[5].elapsed_time(e[6])] for e in ev])
+    st = layer.device_error()
     if st != 0:
         raise RuntimeError(f"device error {L.STATUS.get(st)} in the timed region")
     if clocks:

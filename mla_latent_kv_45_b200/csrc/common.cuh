@@ -31,12 +31,26 @@ template <> __device__ __forceinline__ __nv_bfloat16 st_cast<__nv_bfloat16>(floa
 
 __device__ __forceinline__ void set_error(int *err, int bit) { atomicOr(err, bit); }
 
+// cos / sin of the angle pos * theta in fp64.  The angle is first brought into
+// [-pi, pi] by Cody-Waite reduction with 2 pi split into a double and its
+// rounding remainder (exact enough for any int32 position), so the library
+// sincos only ever sees a small argument.
+__device__ __forceinline__ void rope_cos_sin(int pos, double theta, float &cf, float &sf) {
+  const double a = (double)pos * theta;
+  const double k = rint(a * 0.15915494309189535);      // a / (2 pi), rounded
+  double r = fma(-k, 6.283185307179586, a);             // 2 pi, leading double
+  r = fma(-k, 2.4492935982947064e-16, r);               // 2 pi minus its leading double
+  double s, c;
+  sincos(r, &s, &c);
+  cf = (float)c;
+  sf = (float)s;
+}
+
 // Rotates the pair (x0, x1) by pos * theta_i.
 __device__ __forceinline__ void rope_pair(const RopeParams &rp, int i, int pos, float &x0,
                                           float &x1) {
-  double s, c;
-  sincos((double)pos * rp.theta[i], &s, &c);
-  const float cf = (float)c, sf = (float)s;
+  float cf, sf;
+  rope_cos_sin(pos, rp.theta[i], cf, sf);
   const float a = x0, b = x1;
   x0 = a * cf - b * sf;
   x1 = a * sf + b * cf;

@@ -291,10 +291,10 @@ int sm_count() {
 }  // namespace
 
 int gemm_splits(int m_tiles, int heads, int k_chunks) {
-  // about two resident CTAs per SM, at least 8 K chunks (128 KB of weights) per CTA
+  // about two resident CTAs per SM, at least 4 K chunks (64 KB of weights) per CTA
   const int tiles = m_tiles * heads;
   int s = 2 * sm_count() / tiles;
-  const int max_s = k_chunks / 8 > 0 ? k_chunks / 8 : 1;
+  const int max_s = k_chunks / 4 > 0 ? k_chunks / 4 : 1;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   // no empty split: every split gets ceil(k_chunks / s) chunks but the last

@@ -177,12 +177,7 @@ __global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
   const int b = blockIdx.x;
   const int half = rp.d_rope / 2;
   const int pos = positions[b];
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    double s, c;
-    sincos((double)pos * rp.theta[i], &s, &c);
-    cs[i] = (float)c;
-    sn[i] = (float)s;
-  }
+  for (int i = threadIdx.x; i < half; i += blockDim.x) rope_cos_sin(pos, rp.theta[i], cs[i], sn[i]);
   __syncthreads();
   for (int t = threadIdx.x; t < n_heads * half; t += blockDim.x) {
     const int h = t / half, i = t % half;

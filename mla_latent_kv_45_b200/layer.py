@@ -31,6 +31,11 @@ class DecodeLayer:
             raise ValueError("unsupported dims for the workspace")
         self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         L.mla_workspace_init(self.ws)
+        # the cache append runs on a second stream, beside the query absorption
+        # (the two only meet at the attention), with a workspace of its own
+        self.ws_append = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        L.mla_workspace_init(self.ws_append)
+        self.side = torch.cuda.Stream(device=device)
         H, dt = dims.n_heads, dims.torch_dtype
         self.q_lat = torch.empty(batch, H, dims.d_c + dims.d_rope, dtype=dt, device=device)
         self.z = torch.empty(batch, H, dims.d_c, dtype=dt, device=device)
@@ -39,16 +44,43 @@ class DecodeLayer:
         self.out = torch.empty(batch, d_out, dtype=dt, device=device)
 
     def step(self, cache: L.PagedCache, h: torch.Tensor, positions: torch.Tensor,
-             stream=None) -> torch.Tensor:
+             stream=None, events=None) -> torch.Tensor:
         """Appends h's rows at ``positions`` and returns the layer output.
 
         ``cache.seq_lens`` must already count the new rows (positions + 1).
+        The append runs on a side stream concurrently with the query absorption;
+        the attention waits for both.  ``events`` (7 CUDA events, optional) are
+        recorded around each call: append [0, 1] on the side stream, absorb
+        [2, 3], attention [4, 5] and un-absorption [5, 6] on the main stream.
         """
         w, d = self.w, self.dims
-        L.mla_cache_append(d, cache, h, w["W_DKV"], w["W_KR"], w["gamma"], positions, self.ws,
-                           stream)
+        main = stream if stream is not None else torch.cuda.current_stream()
+        side = self.side
+        side.wait_stream(main)
+        if events:
+            events[0].record(side)
+        L.mla_cache_append(d, cache, h, w["W_DKV"], w["W_KR"], w["gamma"], positions,
+                           self.ws_append, side)
+        if events:
+            events[1].record(side)
+            events[2].record(main)
         L.mla_absorb_q(d, h, w.get("W_DQ"), w["W_UQ"], w["W_QR"], w["W_UK"], positions,
-                       self.q_lat, self.ws, stream)
-        L.mla_decode_attn(d, cache, self.q_lat, self.z, self.lse, self.num_splits, self.ws, stream)
-        L.mla_unabsorb_out(d, self.z, w["W_UV"], w.get("W_O"), self.out, self.ws, stream)
+                       self.q_lat, self.ws, main)
+        if events:
+            events[3].record(main)
+        main.wait_stream(side)
+        if events:
+            events[4].record(main)
+        L.mla_decode_attn(d, cache, self.q_lat, self.z, self.lse, self.num_splits, self.ws, main)
+        if events:
+            events[5].record(main)
+        L.mla_unabsorb_out(d, self.z, w["W_UV"], w.get("W_O"), self.out, self.ws, main)
+        if events:
+            events[6].record(main)
         return self.out
+
+    def device_error(self) -> int:
+        """Synchronises; returns the first nonzero device status of both workspaces."""
+        st = L.mla_get_device_error(self.ws_append, self.side)
+        st2 = L.mla_get_device_error(self.ws)
+        return st if st != 0 else st2

@@ -58,7 +58,7 @@ def test_tiny_fp32_full_step(layout):
     before = cache.pool.clone()
     layer = DecodeLayer(dims, dev_weights(W, wl), wl.batch)
     out = layer.step(cache, dev(h, wl), ipos(prior))
-    assert L.mla_get_device_error(layer.ws) == 0
+    assert layer.device_error() == 0
     ref = oracle.decode_step(h, [pc.rows_f32(b, prior[b]) for b in range(wl.batch)], W, od)
     changed = (cache.pool != before).any(-1).cpu().numpy()
     expect = np.zeros_like(changed)
@@ -92,7 +92,7 @@ def test_tiny_fp32_decode_loop_matches_naive_forward():
     for t in range(T):
         lens.fill_(t + 1)
         outs.append(host(layer.step(cache, dev(hs[:, t], wl), ipos([t] * wl.batch))).copy())
-    assert L.mla_get_device_error(layer.ws) == 0
+    assert layer.device_error() == 0
     for b in range(wl.batch):
         ref = oracle.forward_naive(hs[b], W, od)
         assert_fp32_close(np.stack([o[b] for o in outs]), ref, f"seq {b}")
@@ -224,7 +224,7 @@ def test_bf16_full_step_small_batch():
     cache = dev_cache(pc, prior + 1)
     layer = DecodeLayer(dims, dev_weights(W, wl), wl.batch)
     out = layer.step(cache, dev(h, wl), ipos(prior))
-    assert L.mla_get_device_error(layer.ws) == 0
+    assert layer.device_error() == 0
     ref = oracle.decode_step(h, [pc.rows_f32(b, prior[b]) for b in range(3)], W, oracle_dims(wl))
     assert_bf16_close(host(layer.z), ref["z"], "z")
     assert_bf16_close(host(out), ref["u"], "u")
