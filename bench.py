@@ -105,7 +105,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu_id)],
+                 "-lms", "20", "-i", str(self.gpu_id)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -128,7 +128,9 @@ class ClockSampler:
         if self.proc is None:
             return None
         inside = [s for t, s in self.samples if t0 <= t <= t1]
-        used = inside or [s for _, s in self.samples]
+        # a short timed region may hold no sample: then use the ones within 0.25 s of it
+        near = [s for t, s in self.samples if t0 - 0.25 <= t <= t1 + 0.25]
+        used = inside or near or [s for _, s in self.samples]
         sm, mx, reasons = [], [], set()
         for s in used:
             try:
@@ -142,7 +144,8 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(used), "samples_in_timed_region": len(inside)}
+                "samples": len(used), "samples_in_timed_region": len(inside),
+                "sample_interval_ms": 20}
 
 
 # ---------------------------------------------------------------------------
@@ -355,13 +358,16 @@ def run_mine(args):
 LAUNCHES_PER_STEP = 13
 
 
+ATTN_SOURCES = ("attn_sm100.cu", "kernels_simt.cu", "ptx.cuh", "common.cuh", "kernels.h", "sm100.h")
+
+
 def kernel_revision():
-    """Hash of the CUDA sources (a stored ncu traffic figure is only valid for them)."""
+    """Hash of the sources of the decode-attention call's kernels (plan, attention,
+    merge): a stored ncu traffic figure is only valid for them."""
     import hashlib
-    import glob
     hsh = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "mla_latent_kv_45_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "mla_latent_kv_45_b200", "csrc", name), "rb") as f:
             hsh.update(f.read())
     return hsh.hexdigest()[:16]
 
