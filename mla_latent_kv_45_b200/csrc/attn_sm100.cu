@@ -55,14 +55,8 @@ constexpr int kRow = 576;        // cached values per row
 constexpr int kDc = 512;
 constexpr int kPage = 64;
 constexpr int kOwn = 32;         // rows of a page supplied to the score MMA by each CTA
-#ifndef MLA_ATTN_STAGES
-#define MLA_ATTN_STAGES 3
-#endif
-#ifndef MLA_ATTN_SBUF
-#define MLA_ATTN_SBUF 2
-#endif
-constexpr int kStages = MLA_ATTN_STAGES;
-constexpr int kSBuf = MLA_ATTN_SBUF;   // TMEM score buffers
+constexpr int kStages = 3;
+constexpr int kSBuf = 2;   // TMEM score buffers
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kWarpLoad = 8, kWarpS = 9, kWarpPV = 10, kWarpV = 11;

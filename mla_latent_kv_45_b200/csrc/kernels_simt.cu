@@ -179,15 +179,35 @@ __global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
   const int pos = positions[b];
   for (int i = threadIdx.x; i < half; i += blockDim.x) rope_cos_sin(pos, rp.theta[i], cs[i], sn[i]);
   __syncthreads();
-  for (int t = threadIdx.x; t < n_heads * half; t += blockDim.x) {
-    const int h = t / half, i = t % half;
-    int j0, j1;
-    rope_idx(rp, i, j0, j1);
-    const float *src = qr + ((long)b * n_heads + h) * rp.d_rope;
-    const float x0 = src[j0], x1 = src[j1];
-    T *dst = q_lat + ((long)b * n_heads + h) * (d_c + rp.d_rope) + d_c;
-    dst[j0] = st_cast<T>(x0 * cs[i] - x1 * sn[i]);
-    dst[j1] = st_cast<T>(x0 * sn[i] + x1 * cs[i]);
+  // 8 pairs per thread per round, loads first, so a round costs one memory latency
+  constexpr int kUnroll = 8;
+  const int total = n_heads * half;
+  for (int base = threadIdx.x; base < total; base += blockDim.x * kUnroll) {
+    float x0[kUnroll], x1[kUnroll];
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      const int t = base + k * blockDim.x;
+      if (t < total) {
+        const int h = t / half, i = t % half;
+        int j0, j1;
+        rope_idx(rp, i, j0, j1);
+        const float *src = qr + ((long)b * n_heads + h) * rp.d_rope;
+        x0[k] = __ldg(src + j0);
+        x1[k] = __ldg(src + j1);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      const int t = base + k * blockDim.x;
+      if (t < total) {
+        const int h = t / half, i = t % half;
+        int j0, j1;
+        rope_idx(rp, i, j0, j1);
+        T *dst = q_lat + ((long)b * n_heads + h) * (d_c + rp.d_rope) + d_c;
+        dst[j0] = st_cast<T>(x0[k] * cs[i] - x1[k] * sn[i]);
+        dst[j1] = st_cast<T>(x0[k] * sn[i] + x1[k] * cs[i]);
+      }
+    }
   }
 }
 
@@ -500,33 +520,54 @@ __global__ void combine_kernel(AttnArgs a) {
     if (a.lse) a.lse[(long)b * a.n_heads + h] = M + logf(den);
   }
   __syncthreads();
+  // each thread merges 8 float4 columns at a time: the loads of one piece for
+  // all 8 are issued together, so a block waits for one round trip per piece
   const int nvec = a.d_c / 4;
-  for (int i = threadIdx.x; i < kCombineHeads * nvec; i += blockDim.x) {
-    const int hh = i / nvec, d = (i % nvec) * 4;
-    const int h = h0 + hh;
-    if (h >= a.n_heads) continue;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < pieces; ++j) {
-      const long idx = (long)(pb + j) * a.n_heads + h;
-      float w;
-      if (j < kCombineMaxPieces) {
-        w = wgt[j][hh];
-      } else {  // very long splits: recompute the weight (rare)
-        float M = -INFINITY, den = 0.f;
-        for (int q = 0; q < pieces; ++q) M = fmaxf(M, a.part_m[(long)(pb + q) * a.n_heads + h]);
-        for (int q = 0; q < pieces; ++q) {
-          const long iq = (long)(pb + q) * a.n_heads + h;
-          den += expf(a.part_m[iq] - M) * a.part_l[iq];
-        }
-        w = expf(a.part_m[idx] - M) / den;
-      }
-      const float4 v = *reinterpret_cast<const float4 *>(a.part_O + idx * a.d_c + d);
-      acc.x += w * v.x;
-      acc.y += w * v.y;
-      acc.z += w * v.z;
-      acc.w += w * v.w;
+  const int total = kCombineHeads * nvec;
+  auto weight = [&](int j, int hh) -> float {
+    if (j < kCombineMaxPieces) return wgt[j][hh];
+    const int h = h0 + hh;   // very long splits: recompute the weight (rare)
+    float M = -INFINITY, den = 0.f;
+    for (int q = 0; q < pieces; ++q) M = fmaxf(M, a.part_m[(long)(pb + q) * a.n_heads + h]);
+    for (int q = 0; q < pieces; ++q) {
+      const long iq = (long)(pb + q) * a.n_heads + h;
+      den += expf(a.part_m[iq] - M) * a.part_l[iq];
     }
-    Vec4Out<T>::store(zb + (long)h * a.d_c + d, acc);
+    return expf(a.part_m[(long)(pb + j) * a.n_heads + h] - M) / den;
+  };
+  constexpr int kUnroll = 8;
+  for (int base = threadIdx.x; base < total; base += blockDim.x * kUnroll) {
+    float4 acc[kUnroll];
+    int hh[kUnroll], d[kUnroll];
+    bool ok[kUnroll];
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k) {
+      const int i = base + k * blockDim.x;
+      hh[k] = i / nvec;
+      d[k] = (i % nvec) * 4;
+      ok[k] = i < total && h0 + hh[k] < a.n_heads;
+      acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int j = 0; j < pieces; ++j) {
+      float4 v[kUnroll];
+#pragma unroll
+      for (int k = 0; k < kUnroll; ++k)
+        if (ok[k])
+          v[k] = __ldcg(reinterpret_cast<const float4 *>(
+              a.part_O + ((long)(pb + j) * a.n_heads + h0 + hh[k]) * a.d_c + d[k]));
+#pragma unroll
+      for (int k = 0; k < kUnroll; ++k)
+        if (ok[k]) {
+          const float w = weight(j, hh[k]);
+          acc[k].x += w * v[k].x;
+          acc[k].y += w * v[k].y;
+          acc[k].z += w * v[k].z;
+          acc[k].w += w * v[k].w;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < kUnroll; ++k)
+      if (ok[k]) Vec4Out<T>::store(zb + (long)(h0 + hh[k]) * a.d_c + d[k], acc[k]);
   }
 }
 
