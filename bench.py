@@ -152,7 +152,9 @@ class ClockSampler:
 # our implementation
 # ---------------------------------------------------------------------------
 
-def setup_dist(args):
+def setup_dist(args, backend="nccl"):
+    """Process group from the torchrun environment (one rank per GPU; ``gloo`` for
+    host-only checks).  Sequences are sharded by rank; the data path has no collective."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -160,10 +162,22 @@ def setup_dist(args):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return rank, world, local
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings (the job takes as long as its slowest rank)."""
+    import torch
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
 
 
 def cpu_baseline_sample(wl, W, pc, h, lens, budget_s=20.0):
@@ -290,10 +304,8 @@ def run_mine(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([elapsed, e2e_ms, per_call[:, 2].sum()], device=dev, dtype=torch.float64)
-    if world > 1:
-        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
-    elapsed, e2e_ms, attn_ms_total = times.tolist()
+    elapsed, e2e_ms, attn_ms_total = max_over_ranks([elapsed, e2e_ms, per_call[:, 2].sum()],
+                                                    world, dev)
 
     alg = algorithmic(wl, lens)
     hbm, tf, tf_sus, src = peaks()

@@ -1,0 +1,64 @@
+"""Host-side checks of the multi-rank bench path on CPU: two ``gloo`` ranks.
+
+The decode path shards whole sequences across ranks with no collective; the
+only cross-rank step is the max-over-ranks reduction of the timings, and the
+reference arm runs on rank 0 alone.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import bench
+    from mla_latent_kv_45_b200 import synth
+    import torch.distributed as dist
+    r, w, _ = bench.setup_dist(None, backend="gloo")
+    wl = bench.workload("v2_batch64", r)
+    lens = synth.make_prior_lengths(wl)
+    # every rank reports different timings; all must see the slowest
+    got = bench.max_over_ranks([1.0 + r, 10.0 * (w - r), 3.0], w, "cpu")
+    # the reference arm: rank 0 alone does work
+    calls = []
+    real = bench.workload
+    bench.workload = lambda *a, **k: calls.append(1) or real(*a, **k)
+    if r != 0:
+        bench.run_reference(type("A", (), {"workload": "v2_batch64", "steps": 1, "warmup": 0})())
+    bench.workload = real
+    out.put((r, w, wl.wid, lens.tolist(), got, len(calls)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_and_reduce():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    (r0, w0, wid0, lens0, got0, c0), (r1, w1, wid1, lens1, got1, c1) = res
+    assert (r0, r1, w0, w1) == (0, 1, 2, 2)
+    # distinct shards of sequences with the same shape
+    assert wid0 != wid1 and len(lens0) == len(lens1)
+    assert not np.array_equal(lens0, lens1)
+    # max over ranks, identical on both
+    assert got0 == got1 == [2.0, 20.0, 3.0]
+    # rank 1 returned from the reference arm without building its workload
+    assert c1 == 0
