@@ -224,7 +224,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int part = blockIdx.x >> 1;
-  const PlanHeader hdr = *a.hdr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -263,6 +262,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cluster_sync();  // both CTAs' barriers exist before any remote access
   const uint32_t tmem = bars->tmem_base;
+  // the set-up above overlaps the plan kernel; its results are read from here on
+  grid_dep_wait();
+  grid_dep_launch();
+  const PlanHeader hdr = *a.hdr;
   auto lead = [&](uint64_t *bar) { return mapa(smem_u32(bar), 0); };
 
   TileCursor cur;
@@ -596,8 +599,8 @@ cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s) {
       !make_map(&tm_q, a.q_lat, q_rows, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  attn_sm100_kernel<<<2 * parts, kThreads, kSmemBytes, s>>>(tm_kv, tm_v, tm_q, a, scale_log2);
-  return cudaGetLastError();
+  return launch_pdl(attn_sm100_kernel, dim3(2 * parts), dim3(kThreads), kSmemBytes, s, tm_kv, tm_v,
+                    tm_q, a, scale_log2);
 }
 
 }  // namespace sm100

@@ -56,6 +56,32 @@ __device__ __forceinline__ void rope_pair(const RopeParams &rp, int i, int pos, 
   x1 = a * sf + b * cf;
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl may start
+// while the previous kernel in its stream is still running: it must call
+// grid_dep_wait() before it touches memory that kernel (or an earlier one)
+// writes or reads, and every kernel so launched calls it, which keeps the
+// stream order transitive.  grid_dep_launch() lets the next kernel start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Indices of the two members of RoPE pair i for width d.
 __device__ __forceinline__ void rope_idx(const RopeParams &rp, int i, int &j0, int &j1) {
   if (rp.half) {

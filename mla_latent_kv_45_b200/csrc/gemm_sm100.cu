@@ -118,29 +118,48 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const int tx = kABytes + g.n_pad * 128;
+      // The weights do not depend on the previous kernel: the first stages'
+      // weight tiles are requested before waiting for it, and their
+      // activation tiles (which it may write) after.
+      auto load_a = [&](const Item &it, int i, int st) {
+        const GemmProblem &P = g.p[it.pi];
+        const CUtensorMap *tm_a = it.pi ? &tm_a1 : &tm_a0;
+        uint8_t *a_dst = smem + st * stage_bytes;
+        const int k = (it.kc0 + i) * 64;
+        if (P.a_mn) {
+          // A[m][k] = A2d[head * K + k][m]: two 64-wide MN chunks, 64 K rows each
+          const int y = it.head * P.a_rows_per_head + k;
+          tma_load_2d(a_dst, tm_a, it.m0, y, &bars->full[st]);
+          tma_load_2d(a_dst + kABytes / 2, tm_a, it.m0 + 64, y, &bars->full[st]);
+        } else {
+          tma_load_2d(a_dst, tm_a, k, it.head * P.a_rows_per_head + it.m0, &bars->full[st]);
+        }
+      };
+      int pre = 0;   // chunks whose weight tile was requested before the wait
+      for (int item = item0, c = 0; item < item1 && c < g.stages; ++item) {
+        const Item it = decode_item(g, item);
+        for (int i = 0; i < it.nk && c < g.stages; ++i, ++c, ++pre) {
+          mbar_expect_tx(&bars->full[c], tx);
+          load_a(it, i, c);
+        }
+      }
+      grid_dep_wait();
+      grid_dep_launch();
       int c = 0;
       bool ok = true;
       for (int item = item0; ok && item < item1; ++item) {
         const Item it = decode_item(g, item);
-        const GemmProblem &P = g.p[it.pi];
-        const CUtensorMap *tm_a = it.pi ? &tm_a1 : &tm_a0;
         for (int i = 0; i < it.nk; ++i, ++c) {
           const int st = c % g.stages;
           if (c >= g.stages && !gwait(bars, g.err, &bars->empty[st], ((c / g.stages) - 1) & 1)) {
             ok = false;
             break;
           }
-          uint8_t *a_dst = smem + st * stage_bytes;
-          uint8_t *x_dst = a_dst + kABytes;
+          uint8_t *x_dst = smem + st * stage_bytes + kABytes;
           const int k = (it.kc0 + i) * 64;
-          mbar_expect_tx(&bars->full[st], tx);
-          if (P.a_mn) {
-            // A[m][k] = A2d[head * K + k][m]: two 64-wide MN chunks, 64 K rows each
-            const int y = it.head * P.a_rows_per_head + k;
-            tma_load_2d(a_dst, tm_a, it.m0, y, &bars->full[st]);
-            tma_load_2d(a_dst + kABytes / 2, tm_a, it.m0 + 64, y, &bars->full[st]);
-          } else {
-            tma_load_2d(a_dst, tm_a, k, it.head * P.a_rows_per_head + it.m0, &bars->full[st]);
+          if (c >= pre) {
+            mbar_expect_tx(&bars->full[st], tx);
+            load_a(it, i, st);
           }
           tma_load_2d(x_dst, &tm_x, it.head * g.x_cols_per_head + k, 0, &bars->full[st]);
         }
@@ -232,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Y[n][col_off + m] = sum over splits of part[s][n][m]  (bf16 or fp32 output)
 __global__ void gemm_reduce_kernel(const float *part, int splits, int n_rows, int width,
                                    int part_ld, void *out, long ldy, int out_bf16) {
+  grid_dep_wait();
   const long total = (long)n_rows * width;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
        i += (long)gridDim.x * blockDim.x) {
@@ -366,8 +386,8 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     g.items_per_cta = (items + max_ctas - 1) / max_ctas;
     const int ctas = (items + g.items_per_cta - 1) / g.items_per_cta;
     const size_t smem = (size_t)g.stages * stage_bytes + 256 + 1024;
-    gemm_sm100_kernel<<<ctas, kThreads, smem, s>>>(tm[0], tm[1], tx, g);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(gemm_sm100_kernel, dim3(ctas), dim3(kThreads), smem, s, tm[0], tm[1],
+                               tx, g);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -378,9 +398,8 @@ cudaError_t gemm_reduce(const float *part, int splits, int n, int width, int par
   const long total = (long)n * width;
   int blocks = (int)((total + 255) / 256);
   if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-  gemm_reduce_kernel<<<blocks, 256, 0, s>>>(part, splits, n, width, part_ld, out, ldy,
-                                            out_bf16 ? 1 : 0);
-  return cudaGetLastError();
+  return launch_pdl(gemm_reduce_kernel, dim3(blocks), dim3(256), 0, s, part, splits, n, width,
+                    part_ld, out, ldy, (int)(out_bf16 ? 1 : 0));
 }
 
 }  // namespace sm100

@@ -103,6 +103,7 @@ __global__ void append_finish(const float *xkv, int splits, int batch, int d_c, 
                               int max_pages, int *err) {
   // xkv holds `splits` partial sums [splits][batch][row] of [W_DKV h ; W_KR h]
   extern __shared__ float x[];   // [row]
+  grid_dep_wait();
   const int b = blockIdx.x;
   const int row = d_c + rp.d_rope;
   for (int i = threadIdx.x; i < row; i += blockDim.x) {
@@ -152,10 +153,8 @@ cudaError_t launch_append_finish(const float *xkv, int splits, int batch, int d_
                                  const int32_t *block_table, int max_pages, int *err,
                                  cudaStream_t s) {
   const size_t smem = (d_c + rp.d_rope) * sizeof(float);
-  append_finish<T><<<batch, 256, smem, s>>>(xkv, splits, batch, d_c, rp, gamma, eps, positions,
-                                            pool, num_pages, page_size, block_table, max_pages,
-                                            err);
-  return cudaGetLastError();
+  return launch_pdl(append_finish<T>, dim3(batch), dim3(256), smem, s, xkv, splits, batch, d_c, rp,
+                    gamma, eps, positions, pool, num_pages, page_size, block_table, max_pages, err);
 }
 template cudaError_t launch_append_finish<float>(const float *, int, int, int, const RopeParams &,
                                                  const float *, float, const int32_t *, float *,
@@ -174,6 +173,7 @@ __global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
                        const int32_t *positions, T *q_lat) {
   // the rotation angles pos * theta_i are the same for every head of a sequence
   __shared__ float cs[64], sn[64];
+  grid_dep_wait();
   const int b = blockIdx.x;
   const int half = rp.d_rope / 2;
   const int pos = positions[b];
@@ -214,8 +214,7 @@ __global__ void rope_q(const float *qr, int n_heads, int d_c, RopeParams rp,
 template <class T>
 cudaError_t launch_rope_q(const float *qr, int batch, int n_heads, int d_c, const RopeParams &rp,
                           const int32_t *positions, T *q_lat, cudaStream_t s) {
-  rope_q<T><<<batch, 256, 0, s>>>(qr, n_heads, d_c, rp, positions, q_lat);
-  return cudaGetLastError();
+  return launch_pdl(rope_q<T>, dim3(batch), dim3(256), 0, s, qr, n_heads, d_c, rp, positions, q_lat);
 }
 template cudaError_t launch_rope_q<float>(const float *, int, int, int, const RopeParams &,
                                           const int32_t *, float *, cudaStream_t);
@@ -236,6 +235,8 @@ __global__ void plan_kernel(PlanArgs a) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int tid = threadIdx.x;
+  grid_dep_launch();   // the attention kernel may launch and set up meanwhile
+  grid_dep_wait();
   const long cap = (long)a.max_pages * a.page_size;
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -328,7 +329,8 @@ __global__ void plan_kernel(PlanArgs a) {
 }
 
 cudaError_t launch_plan(const PlanArgs &a, cudaStream_t s) {
-  plan_kernel<<<1, 1024, 0, s>>>(a);
+  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -484,6 +486,7 @@ template <> struct Vec4Out<__nv_bfloat16> {
 
 template <class T>
 __global__ void combine_kernel(AttnArgs a) {
+  grid_dep_wait();
   const int b = blockIdx.x;
   const int h0 = blockIdx.y * kCombineHeads;
   const PlanHeader hdr = *a.hdr;
@@ -574,7 +577,8 @@ __global__ void combine_kernel(AttnArgs a) {
 template <class T>
 cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s) {
   dim3 grid(a.batch, (a.n_heads + kCombineHeads - 1) / kCombineHeads);
-  combine_kernel<T><<<grid, 256, 0, s>>>(a);
+  cudaError_t e = launch_pdl(combine_kernel<T>, grid, dim3(256), 0, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 template cudaError_t launch_combine<float>(const AttnArgs &, cudaStream_t);
