@@ -2,37 +2,42 @@
 // cache rows = 512 latent + 64 shared RoPE key, 64-row pages).
 //
 // The method: every head of a sequence scores the same cached rows, so the
-// 128 absorbed queries q_lat form a dense [128 x 576] operand and each 64-row
-// page is one [64 x 576] tile: S = q_lat . tile^T and O += P . tile[:, :512]
+// 128 absorbed queries q_lat form a dense [128 x 576] operand and the cached
+// rows a dense [rows x 576] one: S = rows . q_lat^T and O += P^T-weighted rows
 // are genuine tensor-core contractions ("从零理解 MLA", 解耦 RoPE absorbed_step:
 // s_c + s_r against the cached [c ; k_R] rows, softmax, z = attn . c;
 // "解耦 RoPE（MLA 下）" §3.3: one k_R shared by all heads, i.e. MQA-shaped).
 //
 // Design (one CTA pair = a 2-CTA cluster per work partition, pair MMAs):
-//  * Scores.  One pair MMA (tcgen05 cta_group::2, M = 256, N = 64, K = 576)
-//    per page: both CTAs supply the same 128 q_lat rows as A (256 columns from
-//    TMEM, 320 from shared memory) and CTA r supplies page rows [32r, 32r+32)
-//    as half of B, so each CTA loads half of the page yet receives the whole
-//    128 x 64 score tile in its TMEM (two score buffers, so the next page's
-//    scores are computed while this one's are read).  Both CTAs then run the
-//    same softmax on identical scores: no score or P crosses between the CTAs.
+//  * A step is 4 pages (256 rows): CTA r holds pages 2r and 2r+1 of the step.
+//  * Scores, rows on TMEM lanes.  One pair MMA chain (tcgen05 cta_group::2,
+//    M = 256 rows, N = 128 heads, K = 576) per step: CTA r supplies its 128
+//    rows as A and q_lat heads [64r, 64r+64) as its half of B, and receives
+//    S^T for its 128 rows x all 128 heads.  No score is computed twice.  The
+//    rows stream through a ring of 64-column chunks, each released as soon as
+//    its four MMAs complete.
+//  * Softmax per head is a reduction over TMEM lanes: each warp reduces its
+//    32 rows with a shuffle transpose (lane L ends with heads 2L, 2L+1), the
+//    four warps of a column half through shared memory, and the pair by an
+//    8-byte st.async exchange per lane.  Both CTAs then hold the same tile
+//    maximum; the running max moves only when it grows by more than 2^8.
 //  * Values.  The fp32 accumulator for 128 heads x 512 latent columns would
-//    fill all of TMEM, so it is held transposed and split: O^T = V^T P^T with
-//    pair MMAs (M = 256 latent columns, two of them per page, N = 128 heads,
-//    K = 64 rows).  CTA r owns latent columns [256b + 128r, +128) for b = 0, 1
-//    (TMEM lane = latent column, TMEM column = head) and supplies heads
-//    [64r, 64r+64) of P as its half of B.
-//  * Once the scores of a page are complete, the stage that held the CTA's 32
-//    rows (read only by the score MMA) is refilled with the page's 64 rows of
-//    this CTA's latent columns (L2 hits: the pair has just streamed the page).
-//  * Softmax: one thread per head (TMEM lane), two warpgroups of 32 rows each,
-//    exp2 domain; the running max moves only when a tile max exceeds it by
-//    more than 2^8, and only then are O^T columns rescaled in TMEM.  Row sums
-//    come from the bf16 P values the MMA consumes.
-//  * Warps 0-7 softmax + epilogue + q_lat TMEM staging; warp 8 loads the
-//    CTA's score rows; warp 9 TMEM allocation, q_lat shared-memory loads and
-//    (even CTA) the score MMAs; warp 10 (even CTA) the P.V MMAs; warp 11 the
-//    latent-column loads for P.V.
+//    fill all of TMEM, so it is held transposed and split: O^T = V^T P with
+//    pair MMAs (M = 256 latent columns, two per page, N = 128 heads, K = 64
+//    rows).  CTA r owns latent columns [256b + 128r, +128) for b = 0, 1 (TMEM
+//    lane = latent column, TMEM column = head) and supplies heads [64r, 64r+64)
+//    of P for all 256 rows of the step as its half of B (MN-major).  It writes
+//    that half for its own rows itself; the partner's rows arrive by one 16 KB
+//    shared-to-shared bulk copy per step (asynchronous proxy, counted on an
+//    mbarrier of the receiving CTA).
+//  * The latent columns a CTA needs for P.V are loaded in their own ring
+//    (mostly L2 hits: the pair has just streamed the rows for the scores).
+//  * Row sums come from the bf16 P values the MMA consumes, reduced like the
+//    maxima (per warp through the shuffle transpose, across the pair at the
+//    end of a sequence piece).
+//  * Warps 0-7 softmax + epilogue; warp 8 loads score rows; warp 9 TMEM
+//    allocation, q_lat loads and (even CTA) the score MMAs; warp 10 (even CTA)
+//    the P.V MMAs; warp 11 the latent-column loads for P.V.
 //  * Partitions come from the plan kernel (equal page counts); a sequence cut
 //    by a partition boundary writes an unnormalised partial that the combine
 //    kernel merges.
@@ -54,56 +59,65 @@ constexpr int kHeads = 128;
 constexpr int kRow = 576;        // cached values per row
 constexpr int kDc = 512;
 constexpr int kPage = 64;
-constexpr int kOwn = 32;         // rows of a page supplied to the score MMA by each CTA
-constexpr int kStages = 3;
-constexpr int kSBuf = 2;   // TMEM score buffers
+constexpr int kStepPages = 4;    // pages per step; CTA r holds step pages 2r, 2r+1
+constexpr int kKSlots = 3;       // score-row chunk ring
+constexpr int kVSlots = 3;       // latent-column chunk ring
 constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kWarpLoad = 8, kWarpS = 9, kWarpPV = 10, kWarpV = 11;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kSleepNs = 20000;   // suspend hint of a waiting thread (woken at completion)
 
-// Shared memory (byte offsets from a 1024-byte aligned base).
-constexpr int kQChunk = kHeads * 128;             // 128 heads x 64 bf16, 128-byte swizzle
-constexpr int kQTmemDims = 2 * (256 - 64 * kSBuf);  // q_lat columns held in TMEM
-constexpr int kQSmem = (kRow - kQTmemDims) / 64;  // the rest, in 64-column shared-memory chunks
-constexpr int kChunk = kOwn * 128;                // 32 rows x 64 bf16
-constexpr int kStageBytes = 9 * kChunk;           // the CTA's 32 rows, all 576 columns
-constexpr int kVBox = kPage * 128;                // 64 rows x 64 latent columns
-constexpr int kVBytes = 4 * kVBox;                // the CTA's 256 latent columns of a page
-constexpr int kPBytes = 64 * 128;                 // P for 64 heads x 64 rows bf16
+// Shared memory (byte offsets from a 1024-byte aligned base).  Every operand
+// tile is made of 64-row x 64-column bf16 boxes with the 128-byte swizzle.
+constexpr int kBox = kPage * 128;           // 8 KB
+constexpr int kQBytes = 9 * kBox;           // q_lat heads [64r, 64r+64), all 576 columns
+constexpr int kKChunk = 2 * kBox;           // the CTA's 128 rows x 64 columns
+constexpr int kVChunk = 2 * kBox;           // one page's 64 rows x 128 latent columns
+constexpr int kPBytes = kStepPages * kBox;  // P: 256 rows x this CTA's 64 heads (MN-major)
+constexpr int kStgBytes = 2 * kBox;         // P of the CTA's rows for the partner's heads
 constexpr int kOffQ = 0;
-constexpr int kOffStage = kOffQ + kQSmem * kQChunk;
-constexpr int kOffP = kOffStage + kStages * kStageBytes;   // two P buffers
-constexpr int kOffRed = kOffP + 2 * kPBytes;      // [2][128] floats: per-warpgroup scratch
-constexpr int kOffAlpha = kOffRed + 1024;         // [128] rescale factors, then [128] row sums
-constexpr int kOffBar = kOffAlpha + 1024;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKSlots * kKChunk;
+constexpr int kOffP = kOffV + kVSlots * kVChunk;
+constexpr int kOffStg = kOffP + kPBytes;
+constexpr int kOffRed = kOffStg + kStgBytes;   // [2 halves][4 warps][64] floats
+constexpr int kOffX = kOffRed + 2048;          // [2 parities][128] the partner's tile maxima
+constexpr int kOffMb = kOffX + 1024;           // [8 warps][64] running max, per warp
+constexpr int kOffAlpha = kOffMb + 2048;       // [128] rescale factors
+constexpr int kOffLsum = kOffAlpha + 512;      // [128] row sums of the pair
+constexpr int kOffLx = kOffLsum + 512;         // [128] the partner's row sums
+constexpr int kOffBar = kOffLx + 512;
 constexpr int kSmemBytes = kOffBar + 512 + 1024;
-static_assert(kVBytes <= kStageBytes, "the latent columns of a page refill its stage");
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0 &&
+                  kOffStg % 1024 == 0,
+              "swizzled tiles start on 1024-byte boundaries");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // TMEM columns
 constexpr uint32_t kTmemO = 0;     // O^T: two blocks of 128 heads (lane = latent column)
-constexpr uint32_t kTmemS = 256;   // S: kSBuf buffers of 64 fp32 columns
-constexpr uint32_t kTmemQ = kTmemS + 64 * kSBuf;   // q_lat columns [0, kQTmemDims) as bf16 pairs
+constexpr uint32_t kTmemS = 256;   // S^T: two buffers of 128 heads (lane = cache row)
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kIdescS = idesc_bf16(256, kPage, 0, 0);   // A = q_lat (K-major), B = rows
-constexpr uint32_t kIdescPV = idesc_bf16(256, 128, 1, 0);    // A = V^T (MN-major), B = P
+constexpr uint32_t kIdescS = idesc_bf16(256, 128, 0, 0);    // A = rows, B = q_lat (K-major)
+constexpr uint32_t kIdescPV = idesc_bf16(256, 128, 1, 1);   // A = V^T, B = P (MN-major)
 constexpr uint16_t kBoth = 3;
 
 struct Bars {
-  uint64_t full[kStages];    // even CTA: the pair's score rows landed (tx, both CTAs)
-  uint64_t empty[kStages];   // P.V of the stage's page complete (pair commit)
-  uint64_t sdone[kStages];   // scores of the stage's page complete (pair commit)
-  uint64_t vland[kStages];   // this CTA's latent columns landed (local tx)
-  uint64_t vready[kStages];  // even CTA: both CTAs' latent columns ready (2 arrivals)
-  uint64_t q_smem;           // even CTA: q_lat shared-memory part of both CTAs (tx)
-  uint64_t q_tmem;           // even CTA: q_lat TMEM part staged in both CTAs (16 warps)
-  uint64_t q_free;           // the segment's last score MMAs complete (pair commit)
-  uint64_t s_full[kSBuf];    // scores in buffer i complete (pair commit)
-  uint64_t s_free[kSBuf];    // even CTA: both CTAs read score buffer i (16 warps)
-  uint64_t p_ready[2];       // even CTA: P written and O^T rescaled in both CTAs (16 warps)
-  uint64_t pv_done[2];       // P.V of the tile using P buffer i complete (pair commit)
+  uint64_t k_full[kKSlots];   // even CTA: both CTAs' row chunks landed (tx)
+  uint64_t k_empty[kKSlots];  // the score MMAs reading the slot complete (pair commit)
+  uint64_t v_land[kVSlots];   // this CTA's latent chunk landed (local tx)
+  uint64_t v_full[kVSlots];   // even CTA: both CTAs' latent chunks ready (2 arrivals)
+  uint64_t v_empty[kVSlots];  // the P.V MMAs reading the slot complete (pair commit)
+  uint64_t q_full;            // even CTA: q_lat halves of both CTAs landed (tx)
+  uint64_t q_free;            // the piece's last score MMAs complete (pair commit)
+  uint64_t s_full[2];         // scores in buffer i complete (pair commit)
+  uint64_t s_free[2];         // even CTA: both CTAs read score buffer i (16 warps)
+  uint64_t mx[2];             // the partner's tile maxima landed (st.async tx)
+  uint64_t p_rx;              // the partner's P rows landed (bulk copy tx)
+  uint64_t p_ready;           // even CTA: P and rescaled O^T of both CTAs ready (16 warps)
+  uint64_t pv_done;           // the step's P.V MMAs complete (pair commit)
+  uint64_t lx;                // the partner's row sums landed (st.async tx)
   uint64_t drain_s, drain_pv;
   uint32_t tmem_base;
   volatile int abort;
@@ -164,9 +178,52 @@ __device__ __forceinline__ bool softmax_any(bool p) {
       : "memory");
   return r != 0;
 }
+// Named barrier over the 128 threads of softmax column half g (warps 4g..4g+3).
+__device__ __forceinline__ void half_sync(int g) {
+  asm volatile("bar.sync %0, 128;" ::"r"(2 + g) : "memory");
+}
 
-// Sequential walk over the tiles (pages) of one partition.
-struct TileCursor {
+struct MaxOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return fmaxf(a, b); }
+};
+struct AddOp {
+  __device__ __forceinline__ float operator()(float a, float b) const { return a + b; }
+};
+
+// One round of the warp transpose-reduction: n values per lane -> n / 2.  The
+// lane whose bit `o` is clear keeps the lower half of its values and receives
+// the partner's lower half; the other keeps and receives the upper half.
+template <int n, int o, class Op>
+__device__ __forceinline__ void xpose_round(float *t, int lane, Op op) {
+  const bool up = lane & o;
+#pragma unroll
+  for (int i = 0; i < n / 2; ++i) {
+    const float keep = up ? t[i + n / 2] : t[i];
+    const float send = up ? t[i] : t[i + n / 2];
+    t[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, o));
+  }
+}
+
+// Reduces 64 per-lane values across the warp's 32 lanes column-wise: on return
+// t[0], t[1] of lane L hold the reductions of columns 2L and 2L+1.
+template <class Op>
+__device__ __forceinline__ void xpose_reduce64(const float (&v)[64], float (&t)[32], int lane,
+                                               Op op) {
+  const bool up = lane & 16;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float keep = up ? v[i + 32] : v[i];
+    const float send = up ? v[i] : v[i + 32];
+    t[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+  xpose_round<32, 8>(t, lane, op);
+  xpose_round<16, 4>(t, lane, op);
+  xpose_round<8, 2>(t, lane, op);
+  xpose_round<4, 1>(t, lane, op);
+}
+
+// Sequential walk over the steps (4 pages) of one partition.
+struct StepCursor {
   SegmentWalker walk;
   Segment seg;
   int lp, nseg;
@@ -178,41 +235,26 @@ struct TileCursor {
     nseg = 0;
   }
   __device__ __forceinline__ void advance(const AttnArgs &a) {
-    if (++lp >= seg.lp1) {
+    lp += kStepPages;
+    if (lp >= seg.lp1) {
       valid = walk.next(a, seg);
       lp = seg.lp0;
       ++nseg;
     }
   }
   __device__ __forceinline__ bool first() const { return lp == seg.lp0; }
-  __device__ __forceinline__ bool last() const { return lp == seg.lp1 - 1; }
-  __device__ __forceinline__ int rows_valid() const { return seg.len - lp * kPage; }
-  __device__ __forceinline__ int page(const AttnArgs &a) const {
-    return a.block_table[(long)seg.b * a.max_pages + lp];
+  __device__ __forceinline__ bool last() const { return lp + kStepPages >= seg.lp1; }
+  // pages of this step that belong to the piece
+  __device__ __forceinline__ int npages() const { return min(kStepPages, seg.lp1 - lp); }
+  // rows of step page j that hold data (>= 1 for j < npages())
+  __device__ __forceinline__ int rows_valid(int j) const { return seg.len - (lp + j) * kPage; }
+  __device__ __forceinline__ int page(const AttnArgs &a, int j) const {
+    return a.block_table[(long)seg.b * a.max_pages + lp + j];
   }
 };
 
-// Stages q_lat[b][h][0:kQTmemDims] into TMEM lane h (bf16 pairs, blocks of 32
-// columns); warpgroup g writes half of the blocks.
-__device__ __forceinline__ void stage_q(const AttnArgs &a, int b, int h, int g, uint32_t taddr) {
-  const uint4 *src = reinterpret_cast<const uint4 *>(
-      reinterpret_cast<const __nv_bfloat16 *>(a.q_lat) + ((long)b * kHeads + h) * kRow);
-  constexpr int kHalfBlocks = kQTmemDims / 128;
-  for (int bb = kHalfBlocks * g; bb < kHalfBlocks * (g + 1); ++bb) {
-    uint32_t v[32];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint4 x = src[bb * 8 + i];
-      v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-    }
-    tmem_st32(taddr + 32 * bb, v);
-  }
-  tmem_wait_st();
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_kv,
-                      const __grid_constant__ CUtensorMap tm_v,
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_rows,
                       const __grid_constant__ CUtensorMap tm_q, const AttnArgs a,
                       const float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
@@ -222,36 +264,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const Ctx ctx{bars, a.err};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
+  const uint32_t peer = rank ^ 1u;
   const bool leader = rank == 0;
   const int part = blockIdx.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->empty[s], 1);
-      mbar_init(&bars->sdone[s], 1);
-      mbar_init(&bars->vland[s], 1);
-      mbar_init(&bars->vready[s], 2);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
     }
-    mbar_init(&bars->q_smem, 1);
-    mbar_init(&bars->q_tmem, 16);
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(&bars->v_land[s], 1);
+      mbar_init(&bars->v_full[s], 2);
+      mbar_init(&bars->v_empty[s], 1);
+    }
+    mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_free, 1);
-    for (int i = 0; i < kSBuf; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->s_free[i], 16);
+      mbar_init(&bars->mx[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars->p_ready[i], 16);
-      mbar_init(&bars->pv_done[i], 1);
-    }
+    mbar_init(&bars->p_rx, 1);
+    mbar_init(&bars->p_ready, 16);
+    mbar_init(&bars->pv_done, 1);
+    mbar_init(&bars->lx, 1);
     mbar_init(&bars->drain_s, 1);
     mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
   if (warp == kWarpLoad && lane == 0) {
-    prefetch_tmap(&tm_kv);
-    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_rows);
     prefetch_tmap(&tm_q);
   }
   if (warp == kWarpS) {
@@ -268,102 +312,140 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const PlanHeader hdr = *a.hdr;
   auto lead = [&](uint64_t *bar) { return mapa(smem_u32(bar), 0); };
 
-  TileCursor cur;
+  StepCursor cur;
   cur.init(a, hdr, part);
 
   if (warp == kWarpLoad) {
-    // ------------------------------- this CTA's 32 rows of each page (score B half)
+    // ------------------------- this CTA's 128 rows of each step, in 64-column chunks
     if (lane == 0) {
-      int tile = 0;
-      for (; cur.valid; cur.advance(a), ++tile) {
-        const int st = tile % kStages;
-        if (tile >= kStages && !wait_bar(ctx, &bars->empty[st], ((tile / kStages) - 1) & 1))
-          break;
-        int page = cur.page(a);
-        if (page < 0 || page >= a.num_pages) {
-          set_error(a.err, kErrRange);
-          a.bad[cur.seg.b] = 1;
-          page = 0;
+      int nk = 0;
+      bool ok = true;
+      for (; cur.valid && ok; cur.advance(a)) {
+        const int np = cur.npages();
+        int pages[2];
+        for (int sp = 0; sp < 2; ++sp) {
+          const int j = 2 * (int)rank + sp;
+          pages[sp] = -1;
+          if (j < np) {
+            int page = cur.page(a, j);
+            if (page < 0 || page >= a.num_pages) {
+              set_error(a.err, kErrRange);
+              a.bad[cur.seg.b] = 1;
+              page = 0;
+            }
+            pages[sp] = page;
+          }
         }
-        if (leader) mbar_expect_tx(&bars->full[st], 2 * kStageBytes);
-        uint8_t *dst = smem + kOffStage + st * kStageBytes;
-        const uint32_t bar = lead(&bars->full[st]);
-        for (int c = 0; c < 9; ++c)
-          tma_load_2d_pair(dst + c * kChunk, &tm_kv, 64 * c, page * kPage + kOwn * rank, bar);
+        for (int c = 0; c < 9; ++c, ++nk) {
+          const int slot = nk % kKSlots;
+          if (nk >= kKSlots && !wait_bar(ctx, &bars->k_empty[slot], ((nk / kKSlots) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          // one 8 KB box per page of the step, from whichever CTA holds it
+          if (leader) mbar_expect_tx(&bars->k_full[slot], np * kBox);
+          uint8_t *dst = smem + kOffK + slot * kKChunk;
+          for (int sp = 0; sp < 2; ++sp)
+            if (pages[sp] >= 0)
+              tma_load_2d_pair(dst + sp * kBox, &tm_rows, 64 * c, pages[sp] * kPage,
+                               lead(&bars->k_full[slot]));
+        }
       }
     }
   } else if (warp == kWarpV) {
-    // --------- after a page's scores: its 64 rows of this CTA's latent columns (P.V A)
-    int tile = 0;
-    for (; cur.valid; cur.advance(a), ++tile) {
-      const int st = tile % kStages;
-      const uint32_t par = (tile / kStages) & 1;
-      if (!wait_bar(ctx, &bars->sdone[st], par)) break;
-      uint8_t *dst = smem + kOffStage + st * kStageBytes;
-      if (lane == 0) {
-        int page = cur.page(a);
-        if (page < 0 || page >= a.num_pages) page = 0;   // flagged by the row loader
-        mbar_expect_tx(&bars->vland[st], kVBytes);
-        // box i = (blk, sub): latent columns 256 blk + 128 r + 64 sub, all 64 rows
-        for (int i = 0; i < 4; ++i)
-          tma_load_2d(dst + i * kVBox, &tm_v, 256 * (i >> 1) + 128 * rank + 64 * (i & 1),
-                      page * kPage, &bars->vland[st]);
-      }
-      if (!wait_bar(ctx, &bars->vland[st], par)) break;
-      const int valid = cur.rows_valid();
+    // ------------- each page's 64 rows of this CTA's 256 latent columns (P.V A operand)
+    int nv = 0, prev_slot = 0, prev_valid = kPage;
+    bool ok = true, pending = false;
+    // hands chunk `idx` (landed) to the P.V issuer; rows past the sequence end
+    // hold arbitrary bytes and are zeroed so that 0 * (stale bytes) cannot reach O
+    auto finish = [&](int slot, int idx, int valid) -> bool {
+      if (!wait_bar(ctx, &bars->v_land[slot], (idx / kVSlots) & 1)) return false;
       if (valid < kPage) {
-        // rows past the sequence end hold arbitrary bytes: zero them so that
-        // 0 * (stale bytes) cannot reach O
-        for (int i = lane; i < (kPage - valid) * 32; i += 32) {
-          const int row = valid + (i >> 5), box = (i >> 3) & 3, piece = i & 7;
-          *reinterpret_cast<uint4 *>(dst + box * kVBox + row * 128 + piece * 16) =
+        uint8_t *dst = smem + kOffV + slot * kVChunk;
+        for (int i = lane; i < (kPage - valid) * 16; i += 32) {
+          const int row = valid + (i >> 4), box = (i >> 3) & 1, piece = i & 7;
+          *reinterpret_cast<uint4 *>(dst + box * kBox + row * 128 + piece * 16) =
               make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(&bars->vready[st]));
-    }
-  } else if (warp == kWarpS) {
-    // ------------- q_lat shared-memory part (both CTAs); the even CTA issues the scores
-    if (lane == 0) {
-      const uint64_t qd = sdesc(smem_u32(smem + kOffQ), 16, 1024, 2);
-      int tile = 0;
-      for (; cur.valid; cur.advance(a), ++tile) {
-        const int st = tile % kStages;
-        if (cur.first()) {
-          // the previous segment's score MMAs must finish before q_lat is replaced
-          if (cur.nseg > 0 && !wait_bar(ctx, &bars->q_free, (cur.nseg - 1) & 1)) break;
-          if (leader) mbar_expect_tx(&bars->q_smem, 2 * kQSmem * kQChunk);
-          for (int c = 0; c < kQSmem; ++c)
-            tma_load_2d_pair(smem + kOffQ + c * kQChunk, &tm_q, kQTmemDims + 64 * c,
-                             cur.seg.b * kHeads, lead(&bars->q_smem));
-          if (leader && (!wait_bar(ctx, &bars->q_smem, cur.nseg & 1) ||
-                         !wait_bar(ctx, &bars->q_tmem, cur.nseg & 1)))
+      if (lane == 0) mbar_arrive_remote(lead(&bars->v_full[slot]));
+      return true;
+    };
+    for (; cur.valid && ok; cur.advance(a)) {
+      const int np = cur.npages();
+      for (int pg = 0; pg < np && ok; ++pg) {
+        int page = cur.page(a, pg);
+        if (page < 0 || page >= a.num_pages) page = 0;   // flagged by the row loader
+        const int valid = min(cur.rows_valid(pg), kPage);
+        for (int blk = 0; blk < 2; ++blk, ++nv) {
+          const int slot = nv % kVSlots;
+          if (nv >= kVSlots && !wait_bar(ctx, &bars->v_empty[slot], ((nv / kVSlots) - 1) & 1)) {
+            ok = false;
             break;
+          }
+          if (lane == 0) {
+            uint8_t *dst = smem + kOffV + slot * kVChunk;
+            mbar_expect_tx(&bars->v_land[slot], kVChunk);
+            // box sub: latent columns 256 blk + 128 r + 64 sub, all 64 rows
+            for (int sub = 0; sub < 2; ++sub)
+              tma_load_2d(dst + sub * kBox, &tm_rows, 256 * blk + 128 * (int)rank + 64 * sub,
+                          page * kPage, &bars->v_land[slot]);
+          }
+          __syncwarp();
+          if (pending && !finish(prev_slot, nv - 1, prev_valid)) {
+            ok = false;
+            break;
+          }
+          prev_slot = slot;
+          prev_valid = valid;
+          pending = true;
+        }
+      }
+    }
+    if (ok && pending) finish(prev_slot, nv - 1, prev_valid);
+  } else if (warp == kWarpS) {
+    // ----------------- q_lat halves (both CTAs); the even CTA issues the score MMAs
+    if (lane == 0) {
+      const uint64_t qd0 = sdesc(smem_u32(smem + kOffQ), 16, 1024, 2);
+      const uint64_t kd0 = sdesc(smem_u32(smem + kOffK), 16, 1024, 2);
+      int step = 0, nk = 0;
+      bool ok = true;
+      for (; cur.valid && ok; cur.advance(a), ++step) {
+        if (cur.first()) {
+          // the previous piece's score MMAs must finish before q_lat is replaced
+          if (cur.nseg > 0 && !wait_bar(ctx, &bars->q_free, (cur.nseg - 1) & 1)) break;
+          if (leader) mbar_expect_tx(&bars->q_full, 2 * kQBytes);
+          for (int c = 0; c < 9; ++c)
+            tma_load_2d_pair(smem + kOffQ + c * kBox, &tm_q, 64 * c,
+                             cur.seg.b * kHeads + 64 * (int)rank, lead(&bars->q_full));
+          if (leader && !wait_bar(ctx, &bars->q_full, cur.nseg & 1)) break;
         }
         if (!leader) continue;
-        if (!wait_bar(ctx, &bars->full[st], (tile / kStages) & 1)) break;
-        // score buffer sb was last used by tile - kSBuf
-        const int sb = tile % kSBuf;
-        if (tile >= kSBuf && !wait_bar(ctx, &bars->s_free[sb], ((tile / kSBuf) - 1) & 1)) break;
-        const uint32_t sd = tmem + kTmemS + 64 * sb;
-        tc_fence_after();
-        // descriptors advance by address >> 4 in their low field (no carry: < 256 KB)
-        const uint64_t kd = sdesc(smem_u32(smem + kOffStage + st * kStageBytes), 16, 1024, 2);
+        const int sb = step & 1;
+        // score buffer sb was last read by the softmax of step - 2
+        if (step >= 2 && !wait_bar(ctx, &bars->s_free[sb], ((step >> 1) - 1) & 1)) break;
+        const uint32_t sd = tmem + kTmemS + 128 * sb;
+        for (int c = 0; c < 9; ++c, ++nk) {
+          const int slot = nk % kKSlots;
+          if (!wait_bar(ctx, &bars->k_full[slot], (nk / kKSlots) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // descriptors advance by address >> 4 in their low field (no carry: < 256 KB)
+          const uint64_t kd = kd0 + (uint64_t)((slot * kKChunk) >> 4);
+          const uint64_t qd = qd0 + (uint64_t)((c * kBox) >> 4);
 #pragma unroll
-        for (int s = 0; s < kQTmemDims / 16; ++s)   // q_lat columns held in TMEM
-          umma_pair_ts(sd, tmem + kTmemQ + 8 * s,
-                       kd + (uint64_t)(((s >> 2) * kChunk + 32 * (s & 3)) >> 4), kIdescS,
-                       s ? 1u : 0u);
-#pragma unroll
-        for (int s = 0; s < 4 * kQSmem; ++s)         // the rest from shared memory
-          umma_pair_ss(sd, qd + (uint64_t)(((s >> 2) * kQChunk + 32 * (s & 3)) >> 4),
-                       kd + (uint64_t)(((kQTmemDims / 64 + (s >> 2)) * kChunk + 32 * (s & 3)) >> 4),
-                       kIdescS, 1u);
+          for (int k = 0; k < 4; ++k)
+            umma_pair_ss(sd, kd + (uint64_t)((32 * k) >> 4), qd + (uint64_t)((32 * k) >> 4),
+                         kIdescS, (c | k) ? 1u : 0u);
+          umma_commit_pair(&bars->k_empty[slot], kBoth);
+        }
+        if (!ok) break;
         if (cur.last()) umma_commit_pair(&bars->q_free, kBoth);
         umma_commit_pair(&bars->s_full[sb], kBoth);
-        umma_commit_pair(&bars->sdone[st], kBoth);
       }
       if (leader) {
         umma_commit_pair(&bars->drain_s, 1);
@@ -373,102 +455,151 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpPV) {
     // ------------------------------------------------- P.V pair MMAs (even CTA)
     if (lane == 0 && leader) {
-      int tile = 0;
-      for (; cur.valid; cur.advance(a), ++tile) {
-        const int st = tile % kStages;
-        const int pb = tile & 1;
-        if (!wait_bar(ctx, &bars->p_ready[pb], (tile >> 1) & 1)) break;
-        if (!wait_bar(ctx, &bars->vready[st], (tile / kStages) & 1)) break;
+      const uint64_t vd0 = sdesc(smem_u32(smem + kOffV), kBox, 1024, 2);
+      const uint64_t pd0 = sdesc(smem_u32(smem + kOffP), kBox, 1024, 2);
+      int step = 0, nv = 0;
+      bool ok = true;
+      for (; cur.valid && ok; cur.advance(a), ++step) {
+        if (!wait_bar(ctx, &bars->p_ready, step & 1)) break;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + kOffStage + st * kStageBytes);
-        const uint64_t pd = sdesc(smem_u32(smem + kOffP + pb * kPBytes), 16, 1024, 2);
+        const int np = cur.npages();
         const bool first = cur.first();
+        for (int pg = 0; pg < np && ok; ++pg) {
+          for (int blk = 0; blk < 2; ++blk, ++nv) {
+            const int slot = nv % kVSlots;
+            if (!wait_bar(ctx, &bars->v_full[slot], (nv / kVSlots) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // A = V^T: two 64-column boxes (8 KB apart), B = P rows of page pg;
+            // both MN-major, 16 rows (2 KB) per MMA
+            const uint64_t vd = vd0 + (uint64_t)((slot * kVChunk) >> 4);
+            const uint64_t pd = pd0 + (uint64_t)((pg * kBox) >> 4);
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          // A = V^T: two 64-column boxes of 64 rows (8 KB apart), MN-major
-          const uint64_t vd = sdesc(v_base + blk * 2 * kVBox, kVBox, 1024, 2);
-#pragma unroll
-          for (int k = 0; k < kPage / 16; ++k)
-            umma_pair_ss(tmem + kTmemO + 128 * blk, vd + (uint64_t)((2048 * k) >> 4),
-                         pd + (uint64_t)((32 * k) >> 4), kIdescPV, (first && k == 0) ? 0u : 1u);
+            for (int k = 0; k < 4; ++k)
+              umma_pair_ss(tmem + kTmemO + 128 * blk, vd + (uint64_t)((2048 * k) >> 4),
+                           pd + (uint64_t)((2048 * k) >> 4), kIdescPV,
+                           (first && pg == 0 && k == 0) ? 0u : 1u);
+            umma_commit_pair(&bars->v_empty[slot], kBoth);
+          }
         }
-        umma_commit_pair(&bars->pv_done[pb], kBoth);
-        umma_commit_pair(&bars->empty[st], kBoth);
+        if (!ok) break;
+        umma_commit_pair(&bars->pv_done, kBoth);
       }
       umma_commit_pair(&bars->drain_pv, 1);
       drain_bar(&bars->drain_pv, 0);
     }
   } else if (warp < 8) {
-    // ----------------------- softmax + epilogue + q_lat staging (warps 0-7)
-    const int g = warp >> 2;                 // warpgroup: page rows [32 g, 32 g + 32)
-    const int quad = warp & 3;
-    const int h = threadIdx.x & 127;         // head == TMEM lane of S
+    // ------------------------------------------- softmax + epilogue (warps 0-7)
+    const int g = warp >> 2;                 // column half: heads [64 g, 64 g + 64)
+    const int quad = warp & 3;               // TMEM lanes [32 quad, 32 quad + 32)
+    const int row = quad * 32 + lane;        // this CTA's row of the step
+    const int sp = quad >> 1;                // ... on the CTA's page sp (step page 2r + sp)
+    const int k = row & 63;                  // ... row k of that page
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float *red = reinterpret_cast<float *>(smem + kOffRed);       // [2][128]
-    float *alpha_s = reinterpret_cast<float *>(smem + kOffAlpha);  // [128]
-    float *lsum = alpha_s + 128;                                   // [128]
-    const bool writes_p = (h >> 6) == (int)rank;   // this CTA supplies P of heads [64r, 64r+64)
-    const int hl = h & 63;
-    float m_run = -INFINITY;     // running max (log2 units), identical in both CTAs
-    float l_part = 0.f;          // this thread's share of the row sum (its 32 rows)
+    float *red = reinterpret_cast<float *>(smem + kOffRed);
+    float *xmax = reinterpret_cast<float *>(smem + kOffX);
+    float *mb = reinterpret_cast<float *>(smem + kOffMb) + warp * 64;
+    float *alpha_s = reinterpret_cast<float *>(smem + kOffAlpha);
+    float *lsum = reinterpret_cast<float *>(smem + kOffLsum);
+    float *lx = reinterpret_cast<float *>(smem + kOffLx);
+    const bool outgoing = g != (int)rank;    // this half of P is the partner's B operand
+    float m0 = -INFINITY, m1 = -INFINITY;    // running max (log2 units) of heads 64g + 2 lane, +1
+    float l0 = 0.f, l1 = 0.f;                // this warp's rows' share of their row sums
 
-    auto produce = [&](int j, const TileCursor &tc) -> bool {
+    // Every softmax thread runs every barrier of a step even after a failed
+    // wait (it then skips the remaining waits and computes garbage), and the
+    // 256 threads agree on stopping by a vote at the end of the step, so no
+    // thread is ever left alone at a named barrier.
+    auto produce = [&](int i, const StepCursor &tc) -> bool {
+      bool ok = true;
       const bool first = tc.first();
-      if (first) {
-        // the previous segment's scores were read, so its score MMAs are complete
-        stage_q(a, tc.seg.b, h, g, tmem + lane_off + kTmemQ);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(lead(&bars->q_tmem));
+      const int sb = i & 1;
+      if (threadIdx.x == 0) {
+        mbar_expect_tx(&bars->mx[sb], 2 * 64 * 4);   // the partner's maxima of step i
+        mbar_expect_tx(&bars->p_rx, kStgBytes);      // the partner's P rows of step i
       }
-      const int sb = j % kSBuf;
-      if (!wait_bar(ctx, &bars->s_full[sb], (j / kSBuf) & 1)) return false;
+      ok = ok && wait_bar(ctx, &bars->s_full[sb], (i >> 1) & 1);
       tc_fence_after();
-      float sv[32];
-      tmem_ld32f(tmem + lane_off + kTmemS + 64 * sb + 32 * g, sv);
+      float v[64];
+      tmem_ld32f(tmem + lane_off + kTmemS + 128 * sb + 64 * g, v);
+      tmem_ld32f(tmem + lane_off + kTmemS + 128 * sb + 64 * g + 32, v + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(lead(&bars->s_free[sb]));
-      const int mine = tc.rows_valid() - 32 * g;     // valid rows among my 32
-      float mx = -INFINITY;
+      const int jp = 2 * (int)rank + sp;
+      const bool valid = jp < tc.npages() && k < tc.rows_valid(jp);
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        sv[k] = k < mine ? sv[k] : -INFINITY;
-        mx = fmaxf(mx, sv[k]);
+      for (int h = 0; h < 64; ++h) v[h] = valid ? v[h] : -INFINITY;
+      // tile max of heads 64g + 2 lane, +1: this warp, the half's four warps, the pair
+      float t[32];
+      xpose_reduce64(v, t, lane, MaxOp());
+      reinterpret_cast<float2 *>(red + (g * 4 + quad) * 64)[lane] = make_float2(t[0], t[1]);
+      half_sync(g);
+      float c0 = -INFINITY, c1 = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 x = reinterpret_cast<const float2 *>(red + (g * 4 + q) * 64)[lane];
+        c0 = fmaxf(c0, x.x);
+        c1 = fmaxf(c1, x.y);
       }
-      softmax_sync();                        // previous readers of red[] are done
-      red[g * 128 + h] = mx;
-      softmax_sync();
-      const float mx_t = fmaxf(red[h], red[128 + h]) * scale_log2;
-      const float m_new = first ? mx_t : (mx_t > m_run + 8.0f ? mx_t : m_run);
-      const float alpha = first ? 1.f : ex2(m_run - m_new);
-      // P (bf16) for my 32 rows; the row sum is taken from the rounded values
-      uint32_t w[16];
-      float add = 0.f;
+      if (quad == 0)
+        st_async_v2(mapa(smem_u32(xmax + sb * 128 + 64 * g + 2 * lane), peer), c0, c1,
+                    mapa(smem_u32(&bars->mx[sb]), peer));
+      ok = ok && wait_bar(ctx, &bars->mx[sb], (i >> 1) & 1);
+      const float2 pm = reinterpret_cast<const float2 *>(xmax + sb * 128 + 64 * g)[lane];
+      const float t0 = fmaxf(c0, pm.x) * scale_log2, t1 = fmaxf(c1, pm.y) * scale_log2;
+      const float n0 = first ? t0 : (t0 > m0 + 8.0f ? t0 : m0);
+      const float n1 = first ? t1 : (t1 > m1 + 8.0f ? t1 : m1);
+      const float a0 = first ? 1.f : ex2(m0 - n0), a1 = first ? 1.f : ex2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      reinterpret_cast<float2 *>(mb)[lane] = make_float2(n0, n1);
+      __syncwarp();
+      // P (bf16) of my row for the half's 64 heads
+      uint32_t w[32];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const float p0 = 2 * q < mine ? ex2(fmaf(sv[2 * q], scale_log2, -m_new)) : 0.f;
-        const float p1 = 2 * q + 1 < mine ? ex2(fmaf(sv[2 * q + 1], scale_log2, -m_new)) : 0.f;
-        w[q] = pack_bf16(p0, p1);
-        add += bf16_lo(w[q]) + bf16_hi(w[q]);
+        const float4 m4 = reinterpret_cast<const float4 *>(mb)[q];
+        w[2 * q] = pack_bf16(ex2(fmaf(v[4 * q], scale_log2, -m4.x)),
+                             ex2(fmaf(v[4 * q + 1], scale_log2, -m4.y)));
+        w[2 * q + 1] = pack_bf16(ex2(fmaf(v[4 * q + 2], scale_log2, -m4.z)),
+                                 ex2(fmaf(v[4 * q + 3], scale_log2, -m4.w)));
       }
-      l_part = first ? add : l_part * alpha + add;
-      m_run = m_new;
-      const int pb = j & 1;
-      if (j >= 2 && !wait_bar(ctx, &bars->pv_done[pb], ((j >> 1) - 1) & 1)) return false;
-      if (writes_p) {
-        // P buffer row hl: 16-byte chunk c (rows 8c..8c+7) at hl*128 + ((c ^ (hl&7)) << 4)
-        uint8_t *row = smem + kOffP + pb * kPBytes + hl * 128;
+      // row sums from the rounded values the MMA consumes
+      {
+        float pr[64];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4 *>(row + (((4 * g + c) ^ (hl & 7)) << 4)) =
-              make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        for (int q = 0; q < 32; ++q) {
+          pr[2 * q] = bf16_lo(w[q]);
+          pr[2 * q + 1] = bf16_hi(w[q]);
+        }
+        xpose_reduce64(pr, t, lane, AddOp());
       }
-      // O^T holds the tiles before j: rescale its head columns when the max moved
-      if (g == 0) alpha_s[h] = alpha;
-      if (softmax_any(alpha != 1.f)) {
-        if (!wait_bar(ctx, &bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) return false;
+      l0 = first ? t[0] : fmaf(l0, a0, t[0]);
+      l1 = first ? t[1] : fmaf(l1, a1, t[1]);
+      // the P buffer (and the staging copy) is free once the previous step's P.V completed
+      if (i > 0) ok = ok && wait_bar(ctx, &bars->pv_done, (i - 1) & 1);
+      // row k of a 64-row box: 16-byte chunk c at k*128 + ((c ^ (k & 7)) << 4)
+      uint8_t *prow = (outgoing ? smem + kOffStg + sp * kBox
+                                : smem + kOffP + (2 * (int)rank + sp) * kBox) + k * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4 *>(prow + ((c ^ (k & 7)) << 4)) =
+            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      fence_proxy_async_smem();              // P -> the MMA / the bulk copy
+      if (outgoing) {
+        half_sync(g);
+        if (quad == 0 && lane == 0)
+          bulk_copy_cta_to_cluster(mapa(smem_u32(smem + kOffP + 2 * (int)rank * kBox), peer),
+                                   smem_u32(smem + kOffStg), kStgBytes,
+                                   mapa(smem_u32(&bars->p_rx), peer));
+      }
+      // O^T holds the steps before i: rescale its head columns when the max moved
+      if (quad == 0) reinterpret_cast<float2 *>(alpha_s + 64 * g)[lane] = make_float2(a0, a1);
+      if (softmax_any(a0 != 1.f || a1 != 1.f)) {
         tc_fence_after();
         const uint32_t ob = tmem + lane_off + kTmemO + 128 * g;   // block g, lane = column
         for (int c = 0; c < 128; c += 32) {
@@ -476,66 +607,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(ob + c, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha_s[c + k]);
+          for (int kk = 0; kk < 32; ++kk)
+            r[kk] = __float_as_uint(__uint_as_float(r[kk]) * alpha_s[c + kk]);
           tmem_st32(ob + c, r);
         }
         tmem_wait_st();
       }
-      fence_proxy_async_smem();              // P -> the MMA
       tc_fence_before();
+      // the partner's rows of this CTA's P half
+      if (warp == 0) ok = ok && wait_bar(ctx, &bars->p_rx, i & 1);
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead(&bars->p_ready[pb]));
-      return true;
+      if (lane == 0) mbar_arrive_remote(lead(&bars->p_ready));
+      return !softmax_any(!ok);
     };
 
-    // ---- end of a segment (tile j was its last): normalise and write O^T
-    auto epilogue = [&](int j, const TileCursor &tc) -> bool {
-      softmax_sync();                        // previous readers of red[] / lsum[] are done
-      red[g * 128 + h] = l_part;
-      softmax_sync();
-      if (g == 0) lsum[h] = red[h] + red[128 + h];
-      if (!wait_bar(ctx, &bars->pv_done[j & 1], (j >> 1) & 1)) return false;
-      softmax_sync();
-      tc_fence_after();
+    // ---- end of a piece (step i was its last): row sums of the pair, normalise, write O^T
+    auto epilogue = [&](int i, const StepCursor &tc) -> bool {
+      bool ok = true;
+      if (threadIdx.x == 0) mbar_expect_tx(&bars->lx, 2 * 64 * 4);
+      reinterpret_cast<float2 *>(red + (g * 4 + quad) * 64)[lane] = make_float2(l0, l1);
+      half_sync(g);
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 x = reinterpret_cast<const float2 *>(red + (g * 4 + q) * 64)[lane];
+        s0 += x.x;
+        s1 += x.y;
+      }
+      if (quad == 0)
+        st_async_v2(mapa(smem_u32(lx + 64 * g + 2 * lane), peer), s0, s1,
+                    mapa(smem_u32(&bars->lx), peer));
+      ok = ok && wait_bar(ctx, &bars->lx, tc.nseg & 1);
+      const float2 px = reinterpret_cast<const float2 *>(lx + 64 * g)[lane];
+      const float f0 = s0 + px.x, f1 = s1 + px.y;   // same sum in both CTAs
+      if (quad == 0) reinterpret_cast<float2 *>(lsum + 64 * g)[lane] = make_float2(f0, f1);
       const int b = tc.seg.b;
       const int pbase = a.part_base[b];
       const bool whole = pbase < 0;
       const int slot_p = whole ? 0 : pbase + (part - tc.seg.s0 / hdr.quota);
-      const int col = 256 * g + 128 * rank + quad * 32 + lane;   // latent column of my lane
+      if (rank == 0 && quad == 0) {
+        const float ln2 = 0.6931471805599453f;
+        const int h0 = 64 * g + 2 * lane;
+        const long ri = (long)b * kHeads + h0;
+        if (whole) {
+          if (a.lse) {
+            a.lse[ri] = (m0 + __log2f(f0)) * ln2;
+            a.lse[ri + 1] = (m1 + __log2f(f1)) * ln2;
+          }
+        } else {
+          a.part_m[(long)slot_p * kHeads + h0] = m0 * ln2;
+          a.part_m[(long)slot_p * kHeads + h0 + 1] = m1 * ln2;
+          a.part_l[(long)slot_p * kHeads + h0] = f0;
+          a.part_l[(long)slot_p * kHeads + h0 + 1] = f1;
+        }
+      }
+      ok = ok && wait_bar(ctx, &bars->pv_done, i & 1);
+      softmax_sync();                        // lsum complete for both halves
+      tc_fence_after();
+      const int col = 256 * g + 128 * (int)rank + quad * 32 + lane;   // latent column of my lane
       const uint32_t ob = tmem + lane_off + kTmemO + 128 * g;
       for (int c = 0; c < 128; c += 32) {
-        float v[32];
-        tmem_ld32f(ob + c, v);
+        float ov[32];
+        tmem_ld32f(ob + c, ov);
         tmem_wait_ld();
         if (whole) {
           __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + (long)b * kHeads * kDc + col;
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            z[(long)(c + k) * kDc] = __float2bfloat16_rn(v[k] / lsum[c + k]);
+          for (int kk = 0; kk < 32; ++kk)
+            z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] / lsum[c + kk]);
         } else {
           float *o = a.part_O + (long)slot_p * kHeads * kDc + col;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[(long)(c + k) * kDc] = v[k];
-        }
-      }
-      if (rank == 0 && g == 0) {
-        const float ln2 = 0.6931471805599453f;
-        const long row_idx = (long)b * kHeads + h;
-        if (whole) {
-          if (a.lse) a.lse[row_idx] = (m_run + __log2f(lsum[h])) * ln2;
-        } else {
-          a.part_m[(long)slot_p * kHeads + h] = m_run * ln2;
-          a.part_l[(long)slot_p * kHeads + h] = lsum[h];
+          for (int kk = 0; kk < 32; ++kk) o[(long)(c + kk) * kDc] = ov[kk];
         }
       }
       tc_fence_before();
-      return true;
+      return !softmax_any(!ok);
     };
 
-    for (int tile = 0; cur.valid; cur.advance(a), ++tile) {
-      if (!produce(tile, cur)) break;
-      if (cur.last() && !epilogue(tile, cur)) break;
+    for (int step = 0; cur.valid; cur.advance(a), ++step) {
+      if (!produce(step, cur)) break;
+      if (cur.last() && !epilogue(step, cur)) break;
     }
   }
 
@@ -591,15 +743,14 @@ cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  CUtensorMap tm_kv, tm_v, tm_q;
+  CUtensorMap tm_rows, tm_q;
   const long pool_rows = (long)a.num_pages * kPage;
   const long q_rows = (long)a.batch * kHeads;
-  if (!make_map(&tm_kv, a.pool, pool_rows, 64, kOwn, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_v, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_q, a.q_lat, q_rows, 64, kHeads, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map(&tm_rows, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&tm_q, a.q_lat, q_rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const float scale_log2 = a.scale * 1.4426950408889634f;
-  return launch_pdl(attn_sm100_kernel, dim3(2 * parts), dim3(kThreads), kSmemBytes, s, tm_kv, tm_v,
+  return launch_pdl(attn_sm100_kernel, dim3(2 * parts), dim3(kThreads), kSmemBytes, s, tm_rows,
                     tm_q, a, scale_log2);
 }
 

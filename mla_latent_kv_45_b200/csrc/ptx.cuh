@@ -394,5 +394,27 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
                : "memory");
 }
 
+// Two floats into another CTA's shared memory, counted (8 bytes) on the
+// destination CTA's mbarrier `mbar`.
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t mbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];"
+      ::"r"(addr), "f"(a), "f"(b), "r"(mbar)
+      : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16, both ends 16-byte aligned) from this
+// CTA's shared memory into another CTA's (cluster address `dst`), counted on
+// the destination CTA's mbarrier `mbar` (cluster address).  The copy runs on
+// the asynchronous proxy: the source must have been made visible to it
+// (fence.proxy.async) by the threads that wrote it.
+__device__ __forceinline__ void bulk_copy_cta_to_cluster(uint32_t dst, uint32_t src,
+                                                         uint32_t bytes, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "r"(src), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+
 }  // namespace ptx
 }  // namespace mla
