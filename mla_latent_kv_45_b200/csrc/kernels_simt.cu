@@ -465,8 +465,9 @@ template cudaError_t launch_attn_simt<float>(const AttnArgs &, int, cudaStream_t
 // z = sum_j w_j O_j / sum_j w_j l_j with w_j = exp(m_j - max_j m_j), and
 // lse = max_j m_j + log(sum_j w_j l_j): the standard merge of partial softmaxes.
 
-constexpr int kCombineHeads = 16;     // heads per block
-constexpr int kCombineMaxPieces = 64; // pieces whose weights are staged in shared memory
+constexpr int kCombineWarps = 8;   // (sequence, head) rows per 256-thread block
+constexpr int kCombinePieces = 4;  // pieces whose loads are in flight together
+constexpr int kCombineVecs = 4;    // float4 columns per lane per pass
 
 template <class T> struct Vec4Out;
 template <> struct Vec4Out<float> {
@@ -484,100 +485,86 @@ template <> struct Vec4Out<__nv_bfloat16> {
   }
 };
 
+// One warp per (sequence, head) row: the lanes reduce the pieces' maxima and
+// weighted row sums with shuffles, then merge the row's columns (4 float4 per
+// lane per pass), with the loads of kCombinePieces pieces in flight together.
+// Pieces are summed in increasing order.
 template <class T>
 __global__ void combine_kernel(AttnArgs a) {
   grid_dep_wait();
-  const int b = blockIdx.x;
-  const int h0 = blockIdx.y * kCombineHeads;
-  const PlanHeader hdr = *a.hdr;
-  T *zb = reinterpret_cast<T *>(a.z) + (long)b * a.n_heads * a.d_c;
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= a.batch * a.n_heads) return;
+  const int b = row / a.n_heads, h = row % a.n_heads;
+  T *zr = reinterpret_cast<T *>(a.z) + (long)row * a.d_c;
   if (a.bad[b]) {
-    for (int i = threadIdx.x; i < kCombineHeads * a.d_c; i += blockDim.x) {
-      const int h = h0 + i / a.d_c;
-      if (h < a.n_heads) zb[(long)h * a.d_c + i % a.d_c] = st_cast<T>(0.f);
-    }
-    if (a.lse)
-      for (int h = h0 + threadIdx.x; h < min(a.n_heads, h0 + kCombineHeads); h += blockDim.x)
-        a.lse[(long)b * a.n_heads + h] = -INFINITY;
+    for (int d = lane; d < a.d_c; d += 32) zr[d] = st_cast<T>(0.f);
+    if (a.lse && lane == 0) a.lse[row] = -INFINITY;
     return;
   }
   const int pb = a.part_base[b];
   if (pb < 0) return;
+  const PlanHeader hdr = *a.hdr;
   const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
   const int pieces = (s1 - 1) / hdr.quota - s0 / hdr.quota + 1;
-  __shared__ float wgt[kCombineMaxPieces][kCombineHeads];
-  // per head: w_j = exp(m_j - M) / sum_j exp(m_j - M) l_j, lse = M + log(sum)
-  for (int hh = threadIdx.x; hh < kCombineHeads; hh += blockDim.x) {
-    const int h = h0 + hh;
-    if (h >= a.n_heads) continue;
-    float M = -INFINITY;
-    for (int j = 0; j < pieces; ++j) M = fmaxf(M, a.part_m[(long)(pb + j) * a.n_heads + h]);
-    float den = 0.f;
-    for (int j = 0; j < pieces; ++j) {
-      const long idx = (long)(pb + j) * a.n_heads + h;
-      den += expf(a.part_m[idx] - M) * a.part_l[idx];
-    }
-    const float inv = 1.f / den;
-    for (int j = 0; j < pieces && j < kCombineMaxPieces; ++j)
-      wgt[j][hh] = expf(a.part_m[(long)(pb + j) * a.n_heads + h] - M) * inv;
-    if (a.lse) a.lse[(long)b * a.n_heads + h] = M + logf(den);
-  }
-  __syncthreads();
-  // each thread merges 8 float4 columns at a time: the loads of one piece for
-  // all 8 are issued together, so a block waits for one round trip per piece
+  const float *pm = a.part_m + (long)pb * a.n_heads + h;   // piece j at pm[j * n_heads]
+  const float *pl = a.part_l + (long)pb * a.n_heads + h;
+  // w_j = exp(m_j - M) / sum_j exp(m_j - M) l_j, lse = M + log(sum)
+  float M = -INFINITY;
+  for (int j = lane; j < pieces; j += 32) M = fmaxf(M, __ldcg(pm + (long)j * a.n_heads));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float den = 0.f;
+  for (int j = lane; j < pieces; j += 32)
+    den += expf(__ldcg(pm + (long)j * a.n_heads) - M) * __ldcg(pl + (long)j * a.n_heads);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  const float inv = 1.f / den;
+  if (a.lse && lane == 0) a.lse[row] = M + logf(den);
   const int nvec = a.d_c / 4;
-  const int total = kCombineHeads * nvec;
-  auto weight = [&](int j, int hh) -> float {
-    if (j < kCombineMaxPieces) return wgt[j][hh];
-    const int h = h0 + hh;   // very long splits: recompute the weight (rare)
-    float M = -INFINITY, den = 0.f;
-    for (int q = 0; q < pieces; ++q) M = fmaxf(M, a.part_m[(long)(pb + q) * a.n_heads + h]);
-    for (int q = 0; q < pieces; ++q) {
-      const long iq = (long)(pb + q) * a.n_heads + h;
-      den += expf(a.part_m[iq] - M) * a.part_l[iq];
-    }
-    return expf(a.part_m[(long)(pb + j) * a.n_heads + h] - M) / den;
-  };
-  constexpr int kUnroll = 8;
-  for (int base = threadIdx.x; base < total; base += blockDim.x * kUnroll) {
-    float4 acc[kUnroll];
-    int hh[kUnroll], d[kUnroll];
-    bool ok[kUnroll];
+  const float4 *src = reinterpret_cast<const float4 *>(a.part_O + ((long)pb * a.n_heads + h) * a.d_c);
+  const long piece_stride = (long)a.n_heads * nvec;   // float4 per piece
+  for (int v0 = 0; v0 < nvec; v0 += 32 * kCombineVecs) {
+    float4 acc[kCombineVecs];
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k) {
-      const int i = base + k * blockDim.x;
-      hh[k] = i / nvec;
-      d[k] = (i % nvec) * 4;
-      ok[k] = i < total && h0 + hh[k] < a.n_heads;
-      acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    for (int j = 0; j < pieces; ++j) {
-      float4 v[kUnroll];
+    for (int q = 0; q < kCombineVecs; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < pieces; j0 += kCombinePieces) {
+      float4 v[kCombinePieces][kCombineVecs];
+      float w[kCombinePieces];
 #pragma unroll
-      for (int k = 0; k < kUnroll; ++k)
-        if (ok[k])
-          v[k] = __ldcg(reinterpret_cast<const float4 *>(
-              a.part_O + ((long)(pb + j) * a.n_heads + h0 + hh[k]) * a.d_c + d[k]));
+      for (int jj = 0; jj < kCombinePieces; ++jj) {
+        const int j = j0 + jj;
+        w[jj] = j < pieces ? expf(__ldcg(pm + (long)j * a.n_heads) - M) * inv : 0.f;
 #pragma unroll
-      for (int k = 0; k < kUnroll; ++k)
-        if (ok[k]) {
-          const float w = weight(j, hh[k]);
-          acc[k].x += w * v[k].x;
-          acc[k].y += w * v[k].y;
-          acc[k].z += w * v[k].z;
-          acc[k].w += w * v[k].w;
+        for (int q = 0; q < kCombineVecs; ++q) {
+          const int vi = v0 + lane + 32 * q;
+          v[jj][q] = (j < pieces && vi < nvec) ? __ldcg(src + j * piece_stride + vi)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < kCombinePieces; ++jj)
+#pragma unroll
+        for (int q = 0; q < kCombineVecs; ++q) {
+          acc[q].x = fmaf(w[jj], v[jj][q].x, acc[q].x);
+          acc[q].y = fmaf(w[jj], v[jj][q].y, acc[q].y);
+          acc[q].z = fmaf(w[jj], v[jj][q].z, acc[q].z);
+          acc[q].w = fmaf(w[jj], v[jj][q].w, acc[q].w);
         }
     }
 #pragma unroll
-    for (int k = 0; k < kUnroll; ++k)
-      if (ok[k]) Vec4Out<T>::store(zb + (long)(h0 + hh[k]) * a.d_c + d[k], acc[k]);
+    for (int q = 0; q < kCombineVecs; ++q) {
+      const int vi = v0 + lane + 32 * q;
+      if (vi < nvec) Vec4Out<T>::store(zr + 4 * vi, acc[q]);
+    }
   }
 }
 
 template <class T>
 cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s) {
-  dim3 grid(a.batch, (a.n_heads + kCombineHeads - 1) / kCombineHeads);
-  cudaError_t e = launch_pdl(combine_kernel<T>, grid, dim3(256), 0, s, a);
+  const int rows = a.batch * a.n_heads;
+  const dim3 grid((rows + kCombineWarps - 1) / kCombineWarps);
+  cudaError_t e = launch_pdl(combine_kernel<T>, grid, dim3(32 * kCombineWarps), 0, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
