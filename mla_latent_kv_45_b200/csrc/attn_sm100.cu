@@ -31,7 +31,8 @@
 //    shared-to-shared bulk copy per step (asynchronous proxy, counted on an
 //    mbarrier of the receiving CTA).
 //  * The latent columns a CTA needs for P.V are loaded in their own ring
-//    (mostly L2 hits: the pair has just streamed the rows for the scores).
+//    (mostly L2 hits: the pair has just streamed the rows for the scores; the
+//    row loads carry an evict-last L2 policy and these reloads evict-first).
 //  * Row sums come from the bf16 P values the MMA consumes, reduced like the
 //    maxima (per warp through the shuffle transpose, across the pair at the
 //    end of a sequence piece).
@@ -345,10 +346,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // one 8 KB box per page of the step, from whichever CTA holds it
           if (leader) mbar_expect_tx(&bars->k_full[slot], np * kBox);
           uint8_t *dst = smem + kOffK + slot * kKChunk;
+          // evict-last: the rows are read again (latent columns) for P.V shortly after
           for (int sp = 0; sp < 2; ++sp)
             if (pages[sp] >= 0)
-              tma_load_2d_pair(dst + sp * kBox, &tm_rows, 64 * c, pages[sp] * kPage,
-                               lead(&bars->k_full[slot]));
+              tma_load_2d_pair_hint(dst + sp * kBox, &tm_rows, 64 * c, pages[sp] * kPage,
+                                    lead(&bars->k_full[slot]), l2_policy_evict_last());
         }
       }
     }
@@ -388,10 +390,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             uint8_t *dst = smem + kOffV + slot * kVChunk;
             mbar_expect_tx(&bars->v_land[slot], kVChunk);
-            // box sub: latent columns 256 blk + 128 r + 64 sub, all 64 rows
+            // box sub: latent columns 256 blk + 128 r + 64 sub, all 64 rows; the last
+            // read of these bytes, so evict-first
             for (int sub = 0; sub < 2; ++sub)
-              tma_load_2d(dst + sub * kBox, &tm_rows, 256 * blk + 128 * (int)rank + 64 * sub,
-                          page * kPage, &bars->v_land[slot]);
+              tma_load_2d_hint(dst + sub * kBox, &tm_rows, 256 * blk + 128 * (int)rank + 64 * sub,
+                               page * kPage, &bars->v_land[slot], l2_policy_evict_first());
           }
           __syncwarp();
           if (pending && !finish(prev_slot, nv - 1, prev_valid)) {
