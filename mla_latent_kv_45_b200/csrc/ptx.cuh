@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiled loads, the
 // tcgen05 tensor-core path (TMEM allocation, MMA, commit, TMEM loads/stores)
-// and cluster shared memory.  No multicast form is used anywhere.
+// and cluster shared memory (st.async, bulk copies), L2 cache policies.  No
+// multicast form is used anywhere.
 #pragma once
 
 #include <cuda.h>
@@ -65,19 +66,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-// Arrive (release at cluster scope) on a barrier in another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
-// Relaxed remote arrive: orders nothing, only counts (for "slot consumed" signals
-// whose reads have already completed).
-__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -140,14 +128,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Asks L2 to fetch [p, p + bytes) from global memory (no shared memory involved).
-// p 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
@@ -231,17 +211,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : "r"(taddr));
 }
 
-// 16 consecutive TMEM columns of this thread's lane as fp32 (warp-collective).
-__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float *v) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
-        "=f"(v[7]), "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]),
-        "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
-      : "r"(taddr));
-}
-
 // Same as tmem_ld32, delivering fp32 values straight into v[0..31].
 __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float *v) {
   asm volatile(
@@ -269,26 +238,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       "r"(v[29]), "r"(v[30]), "r"(v[31]));
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-      "r"(v[15]));
-}
-
-// tcgen05.mma with the A operand in tensor memory (row i of A in lane i, two
-// 16-bit elements per 32-bit column, the lower k in the low half).
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
 // ------------------------------------------------- CTA-pair (cta_group::2) forms
 // One MMA issued by the even CTA of a 2-CTA cluster computes M = 256 rows: each
 // CTA supplies 128 rows of A (TMEM or shared memory, same address in both) and
@@ -306,15 +255,6 @@ __device__ __forceinline__ void tmem_alloc_pair(uint32_t *slot_smem, uint32_t nc
 __device__ __forceinline__ void tmem_dealloc_pair(uint32_t base, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(ncols)
                : "memory");
-}
-
-__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -363,37 +303,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 
 // ---------------------------------------------------------------- DSMEM
 
-// Asynchronous 16-byte store into another CTA's shared memory; on arrival it
-// completes 16 bytes of the transaction count of the mbarrier `mbar` (also in
-// the destination CTA), so the sender never waits or fences.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
-                                            uint32_t mbar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-      ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(mbar)
-      : "memory");
-}
-
-__device__ __forceinline__ void st_async_v4u(uint32_t addr, uint4 v, uint32_t mbar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-      ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(mbar)
-      : "memory");
-}
-
-__device__ __forceinline__ void st_async_f32(uint32_t addr, float a, uint32_t mbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
-               ::"r"(addr), "r"(__float_as_uint(a)), "r"(mbar)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c,
-                                              float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
-
 // Two floats into another CTA's shared memory, counted (8 bytes) on the
 // destination CTA's mbarrier `mbar`.
 __device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t mbar) {
@@ -416,7 +325,9 @@ __device__ __forceinline__ void bulk_copy_cta_to_cluster(uint32_t dst, uint32_t 
       : "memory");
 }
 
-// L2 eviction policies for cache-hinted loads.
+// ------------------------------------------------------ L2 cache policies
+
+// L2 eviction policies for cache-hinted loads (every access of the load gets it).
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -428,6 +339,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return p;
 }
 
+// tma_load_2d / tma_load_2d_pair with an L2 eviction policy for the loaded lines.
 __device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, int x, int y,
                                                  uint64_t *bar, uint64_t policy) {
   asm volatile(
