@@ -319,14 +319,7 @@ def run_mine(args):
         achieved, peak, unit = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9, hbm, "GB/s"
     else:
         achieved, peak, unit = alg["attn_flops"] / (attn_ms / 1e3) / 1e12, tf, "TFLOP/s"
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", "attn_traffic.json")
-    if os.path.exists(tfile):
-        with open(tfile) as f:
-            tinfo = json.load(f)
-        if tinfo.get("workload") == wl.name.split("+")[0] and tinfo.get("kernel_rev") == \
-                kernel_revision():
-            traffic = tinfo.get("dram_bytes_per_launch")
+    traffic = stored_traffic(wl.name.split("+")[0])
     step_t = max(alg["step_bytes"] / (hbm * 1e9), alg["step_flops"] / (tf * 1e12))
     h2d = (hd.numel() * hd.element_size() + pos.numel() * 4 + cache.seq_lens.numel() * 4)
     d2h = layer.out.numel() * layer.out.element_size()
@@ -371,6 +364,19 @@ LAUNCHES_PER_STEP = 13
 
 
 ATTN_SOURCES = ("attn_sm100.cu", "kernels_simt.cu", "ptx.cuh", "common.cuh", "kernels.h", "sm100.h")
+
+
+def stored_traffic(workload, tfile=None):
+    """DRAM bytes per decode-attention call from the committed ncu capture, or
+    None when the capture is for another workload or for other kernel sources."""
+    tfile = tfile or os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(tfile):
+        return None
+    with open(tfile) as f:
+        tinfo = json.load(f)
+    if tinfo.get("workload") != workload or tinfo.get("kernel_rev") != kernel_revision():
+        return None
+    return tinfo.get("dram_bytes_per_launch")
 
 
 def kernel_revision():

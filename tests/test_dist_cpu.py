@@ -62,3 +62,17 @@ def test_two_gloo_ranks_shard_and_reduce():
     assert got0 == got1 == [2.0, 20.0, 3.0]
     # rank 1 returned from the reference arm without building its workload
     assert c1 == 0
+
+
+def test_stored_traffic_only_for_the_captured_sources(tmp_path):
+    import json
+    import bench
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps({"workload": "v2_batch64", "kernel_rev": bench.kernel_revision(),
+                             "dram_bytes_per_launch": 123}))
+    assert bench.stored_traffic("v2_batch64", str(f)) == 123
+    assert bench.stored_traffic("v2_step128", str(f)) is None
+    f.write_text(json.dumps({"workload": "v2_batch64", "kernel_rev": "0" * 16,
+                             "dram_bytes_per_launch": 123}))
+    assert bench.stored_traffic("v2_batch64", str(f)) is None
+    assert bench.stored_traffic("v2_batch64", str(tmp_path / "missing.json")) is None
