@@ -133,6 +133,22 @@ def test_bf16_attn_ragged(splits):
         np.testing.assert_allclose(lh[b], lr, atol=2e-3, rtol=0)
 
 
+@pytest.mark.parametrize("splits", [0, 3, 16])
+def test_bf16_attn_step_tails(splits):
+    """1 to 9 pages with a one-row and a full last page: the attention takes pages
+    four at a time (two per CTA of the pair), so this covers every shape of a
+    piece's last step, whole and cut into partitions."""
+    lens = np.array([64 * n + r for n in range(9) for r in (1, 64)])
+    wl, pc, q, z, lse, st = attn_case(lens, splits)
+    assert st == 0
+    od = oracle_dims(wl)
+    zh, lh = host(z), host(lse)
+    for b, Lb in enumerate(lens):
+        zr, lr = oracle.attend_latent(q[b], pc.rows_f32(b, Lb), od)
+        assert_bf16_close(zh[b], zr, f"z seq {b} len {Lb}")
+        np.testing.assert_allclose(lh[b], lr, atol=2e-3, rtol=0)
+
+
 def test_bf16_attn_split_and_page_order_invariance():
     lens = np.array([900, 5, 300, 2000])
     _, _, _, z1, l1, _ = attn_case(lens, 1)
