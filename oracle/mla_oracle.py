@@ -27,6 +27,8 @@ Pins (tests/test_oracle_pins.py) -- every function below is pinned:
                       equals the unsplit softmax.
 * ``unabsorb``        absorption identity ``W_UV,i z_i == o_i``; brute force.
 * ``forward_naive``   causal brute force; equals the step-by-step absorbed loop.
+* ``gather_rows``     rows scattered one by one into a shuffled pool by the
+                      layout's definition come back in logical order.
 """
 
 from __future__ import annotations

@@ -61,11 +61,6 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def pool_rows(cache: L.PagedCache, bt: np.ndarray, b: int, length: int, page_size: int):
-    pool = host(cache.pool)
-    return oracle.gather_rows(pool, bt, b, length, page_size)
-
-
 def metrics(g, r):
     g = np.asarray(g, np.float64)
     r = np.asarray(r, np.float64)

@@ -478,3 +478,45 @@ def test_pins_catch_absorption_mistakes():
     assert _fails(check_absorption, absorb_q, _attend_no_rope_part, unabsorb)
     assert _fails(check_absorption, absorb_q, attend_latent, _unabsorb_transposed)
     assert _fails(check_attend_special, _attend_wrong_scale)
+
+
+# ---------------------------------------------------------------------------
+# Paged-cache gather: row s of sequence b sits at page bt[b][s // P], slot s % P
+# ---------------------------------------------------------------------------
+
+def check_gather(gather_fn):
+    """Scatter known rows into a shuffled pool one at a time (the layout's
+    definition, written as a loop), then the gather must give them back in
+    logical order, for ragged lengths and for a length that ends mid-page."""
+    rng = _r(77)
+    P, width, pages = 4, 5, 11
+    perm = rng.permutation(pages)
+    bt = np.full((2, 4), -1, dtype=np.int64)
+    bt[0, :3] = perm[:3]
+    bt[1, :4] = perm[3:7]
+    pool = np.full((pages, P, width), np.nan)
+    rows = {0: rng.standard_normal((10, width)), 1: rng.standard_normal((13, width))}
+    for b, r in rows.items():
+        for s in range(len(r)):
+            pool[bt[b, s // P], s % P] = r[s]
+    for b, r in rows.items():
+        for n in (1, P, P + 1, len(r)):
+            got = gather_fn(pool, bt, b, n, P)
+            assert got.shape == (n, width)
+            assert np.array_equal(got, r[:n])
+
+
+def test_gather_rows_pin():
+    check_gather(oracle.gather_rows)
+
+
+def test_pins_catch_gather_mistakes():
+    def slot_swapped(pool, bt, b, n, P):   # page and slot indices exchanged
+        idx = np.arange(n)
+        return np.asarray(pool)[np.asarray(bt)[b][idx % P], idx // P]
+
+    def pool_order(pool, bt, b, n, P):     # ignores the page table
+        return np.asarray(pool).reshape(-1, pool.shape[-1])[:n]
+
+    for bad in (slot_swapped, pool_order):
+        assert _fails(check_gather, bad)

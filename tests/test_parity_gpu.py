@@ -106,18 +106,22 @@ V2R = synth.reduced(synth.V2_BATCH64, "v2_ragged", 20, 6, 0, 0)
 RAGGED = np.array([1, 63, 64, 65, 700, 129])
 
 
+def run_attn(wl, pc, q, lens, splits=0):
+    """mla_decode_attn on host inputs; returns (z, lse, device status)."""
+    dims = lib_dims(wl)
+    cache = dev_cache(pc, lens)
+    ws = new_ws(dims, wl.batch, splits=splits)
+    z = torch.empty(wl.batch, wl.n_heads, wl.d_c, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(wl.batch, wl.n_heads, dtype=torch.float32, device="cuda")
+    L.mla_decode_attn(dims, cache, dev(q, wl), z, lse, splits, ws)
+    return z, lse, L.mla_get_device_error(ws)
+
+
 def attn_case(lens, splits=0, wl=V2R, shuffle=True):
     wl = dataclasses.replace(wl, batch=len(lens), new_tokens=0, shuffle_pages=shuffle)
     pc = synth.make_paged_cache(wl, np.asarray(lens), spare_pages=2)
     q = synth.make_q_lat(wl)
-    dims = lib_dims(wl)
-    cache = dev_cache(pc, lens)
-    ws = new_ws(dims, wl.batch, splits=splits)
-    qd = dev(q, wl)
-    z = torch.empty(wl.batch, wl.n_heads, wl.d_c, dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty(wl.batch, wl.n_heads, dtype=torch.float32, device="cuda")
-    L.mla_decode_attn(dims, cache, qd, z, lse, splits, ws)
-    st = L.mla_get_device_error(ws)
+    z, lse, st = run_attn(wl, pc, q, lens, splits)
     return wl, pc, q, z, lse, st
 
 
@@ -336,3 +340,152 @@ def test_bf16_attn_long_sampled():
         zr, lr = oracle.attend_latent(q[b], pc.rows_f32(b, lens[b]), od)
         assert_bf16_close(zh[b], zr, f"seq {b}")
         np.testing.assert_allclose(lh[b], lr, atol=2e-3, rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# Softmax paths of the attention kernel
+# ---------------------------------------------------------------------------
+#
+# The kernel takes a piece of a sequence in steps of STEP_ROWS rows and keeps a
+# running maximum in log2 units that moves only when a step's maximum exceeds it
+# by more than RESCALE_LOG2; only then is the accumulated O rescaled.
+
+STEP_ROWS = 256
+RESCALE_LOG2 = 8.0
+SOFTMAX_LENS = np.array([1, 63, 65, 256, 257, 700, 3000, 5000])
+
+
+def _set_rows(pc, b, rows):
+    idx = np.arange(len(rows))
+    pc.pool[pc.block_table[b][idx // pc.page_size], idx % pc.page_size] = synth.bf16_bits(rows)
+
+
+def _ramp_case():
+    """k_R of row s grows from x1 to x16 along each sequence, c stays N(0, 1):
+    the position score, and with it each head's running maximum, rises step
+    after step by far more than 2^8, while z stays a mean of N(0, 1) rows."""
+    lens = SOFTMAX_LENS
+    wl = dataclasses.replace(V2R, batch=len(lens), new_tokens=0)
+    pc = synth.make_paged_cache(wl, lens, spare_pages=2)
+    for b, Lb in enumerate(lens):
+        rows = pc.rows_f32(b, Lb).copy()
+        rows[:, 512:] *= (1.0 + 15.0 * np.arange(Lb) / max(Lb - 1, 1))[:, None]
+        _set_rows(pc, b, rows)
+    return wl, pc, synth.make_q_lat(wl)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3, 16])
+def test_bf16_attn_rescale_path(splits):
+    wl, pc, q, = _ramp_case()
+    od = oracle_dims(wl)
+    # the inputs do drive the rescale: for every head of the long sequences the
+    # maximum over the whole sequence exceeds the first step's by more than 2^8
+    # (in log2 units), so an unsplit piece must move its running max at least once
+    for b in (6, 7):
+        lg = (q[b].astype(np.float64) @ pc.rows_f32(b, SOFTMAX_LENS[b]).T) * od.scale / np.log(2)
+        assert np.all(lg.max(1) - lg[:, :STEP_ROWS].max(1) > 4 * RESCALE_LOG2)
+    z, lse, st = run_attn(wl, pc, q, SOFTMAX_LENS, splits)
+    assert st == 0
+    zh, lh = host(z), host(lse)
+    for b, Lb in enumerate(SOFTMAX_LENS):
+        zr, lr = oracle.attend_latent(q[b], pc.rows_f32(b, Lb), od)
+        assert_bf16_close(zh[b], zr, f"z seq {b} len {Lb}")
+        # a near one-hot softmax: the dominant row's bf16 P carries up to 2^-9
+        # relative error, ln(1 + 2^-9) = 1.95e-3 in lse
+        np.testing.assert_allclose(lh[b], lr, atol=4e-3, rtol=0)
+
+
+@pytest.mark.parametrize("splits", [0, 3, 16])
+def test_bf16_attn_one_dominant_row(splits):
+    """Every head shares one q_R; a planted row with k_R = 10 q_R scores ~40 nats
+    above the rest, so z is that row's latent c: exactly, after the bf16 store."""
+    lens = SOFTMAX_LENS
+    wl = dataclasses.replace(V2R, batch=len(lens), new_tokens=0)
+    pc = synth.make_paged_cache(wl, lens, spare_pages=2)
+    q = synth.make_q_lat(wl).copy()
+    u = q[:, 0, 512:].copy()
+    q[:, :, 512:] = u[:, None, :]
+    # first row, last row, a page's middle, the first row of a later step, ...
+    where = [0, 62, 64, 255, 256, 699, 1536, 4999]
+    for b, (Lb, p) in enumerate(zip(lens, where)):
+        assert p < Lb
+        rows = pc.rows_f32(b, Lb).copy()
+        rows[p, 512:] = synth.round_bf16(10.0 * u[b])
+        _set_rows(pc, b, rows)
+    z, lse, st = run_attn(wl, pc, q, lens, splits)
+    assert st == 0
+    zh = host(z)
+    od = oracle_dims(wl)
+    for b, (Lb, p) in enumerate(zip(lens, where)):
+        rows = pc.rows_f32(b, Lb)
+        assert np.array_equal(zh[b], np.broadcast_to(rows[p, :512], zh[b].shape)), b
+        zr, lr = oracle.attend_latent(q[b], rows, od)
+        assert_bf16_close(zh[b], zr, f"seq {b}")
+        np.testing.assert_allclose(host(lse)[b], lr, atol=2e-3, rtol=0)
+
+
+@pytest.mark.parametrize("splits", [0, 3, 16])
+def test_bf16_attn_equal_scores(splits):
+    """q_lat = 0: every score is 0, so z is the plain mean of the sequence's c rows
+    (any row past the end that leaked in would move it) and lse = ln L."""
+    lens = SOFTMAX_LENS
+    wl = dataclasses.replace(V2R, batch=len(lens), new_tokens=0)
+    pc = synth.make_paged_cache(wl, lens, spare_pages=2)
+    # fill the unused slots of the last pages with large values
+    for b, Lb in enumerate(lens):
+        for s in range(Lb, -(-Lb // 64) * 64):
+            pc.pool[pc.block_table[b][s // 64], s % 64] = synth.bf16_bits(np.full(576, 1e4))
+    q = np.zeros((len(lens), 128, 576), np.float32)
+    z, lse, st = run_attn(wl, pc, q, lens, splits)
+    assert st == 0
+    zh, lh = host(z), host(lse)
+    for b, Lb in enumerate(lens):
+        mean = pc.rows_f32(b, Lb)[:, :512].astype(np.float64).mean(0)
+        assert_bf16_close(zh[b], np.broadcast_to(mean, zh[b].shape), f"seq {b}")
+        np.testing.assert_allclose(lh[b], np.log(Lb), rtol=1e-6, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Whole decode steps at the full workload sizes (z and the layer output u)
+# ---------------------------------------------------------------------------
+
+def full_step(wl, prior, W, pc, h):
+    cache = dev_cache(pc, prior + 1)
+    layer = DecodeLayer(lib_dims(wl), dev_weights(W, wl), wl.batch)
+    out = layer.step(cache, dev(h, wl), ipos(prior))
+    assert layer.device_error() == 0
+    # absorbed form of the oracle (pinned equal to the un-absorbed one)
+    ref = oracle.decode_step(h, [pc.rows_f32(b, prior[b]) for b in range(wl.batch)], W,
+                             oracle_dims(wl), unabsorbed=False)
+    assert_bf16_close(host(layer.q_lat), ref["q_lat"], "q_lat")
+    zh = host(layer.z)
+    for b in range(wl.batch):
+        assert_bf16_close(zh[b], ref["z"][b], f"z seq {b}")
+    np.testing.assert_allclose(host(layer.lse), ref["lse"], atol=2e-3, rtol=0)
+    assert_bf16_close(host(out), ref["u"], "u")
+
+
+def test_bf16_full_step_v2_single():
+    """batch 1, 4096 cached rows + the new one, W_DQ .. W_O: the smallest grid."""
+    wl = synth.V2_SINGLE
+    prior = synth.make_prior_lengths(wl)
+    full_step(wl, prior, synth.make_weights(wl), synth.make_paged_cache(wl, prior),
+              synth.make_hidden(wl))
+
+
+def test_bf16_full_step_v2_step128():
+    """batch 128, 2048 cached rows + the new one each, the whole layer step."""
+    wl = synth.V2_STEP128
+    prior = synth.make_prior_lengths(wl)
+    full_step(wl, prior, synth.make_weights(wl), synth.make_paged_cache(wl, prior),
+              synth.make_hidden(wl))
+
+
+def test_bf16_full_step_bench_inputs():
+    """The decode step on exactly the inputs bench.py times (rank 0's shard of
+    batch 64, cached rows U[1024, 8192] + 1, shuffled pages)."""
+    import bench
+    wl = bench.workload("v2_batch64", 0)
+    prior = synth.make_prior_lengths(wl)
+    full_step(wl, prior, synth.make_weights(wl), synth.make_paged_cache(wl, prior),
+              synth.make_hidden(wl))
