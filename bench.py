@@ -3,9 +3,10 @@
 
 One step = one pass of the whole decode hot path of one layer for a batch:
 ``mla_cache_append`` (W_DKV + RMSNorm, W_KR + RoPE, paged write) ->
-``mla_absorb_q`` (W_DQ, W_UQ, W_QR + RoPE, W_UK absorption) ->
+``mla_absorb_q`` (W_DQ, then W_UQ + W_QR + RoPE + W_UK absorption per head) ->
 ``mla_decode_attn`` (latent attention over every cached row, split-KV merge) ->
-``mla_unabsorb_out`` (W_UV, W_O).
+``mla_unabsorb_out`` (W_UV, W_O).  The long-context workload (``v2_long``,
+131072 rows per sequence) times the attention call alone.
 
 Metric: cached-token x heads per second (sum over sequences of the rows each
 new token attends to, times 128 heads, per second), plus the attention call's
@@ -15,8 +16,14 @@ the workload's shape; weights N(0, 0.02^2).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
-Multi-GPU (torchrun): data-parallel over sequences, each rank its own batch
-(weak scaling), no collective on the data path; timing is the max over ranks.
+The timed region replays the step captured once as a CUDA graph (the same
+launches the eager calls make); a second, eager pass records per-call CUDA
+events for the breakdown and the attention call's roofline, and a third pass
+measures the end-to-end number through the Python API with host buffers.
+
+Multi-GPU: ``--gpus N`` starts N ranks on this node (one per GPU, NCCL),
+data-parallel over sequences, each rank its own batch (weak scaling), no
+collective on the data path; timing is the max over ranks.
 """
 
 from __future__ import annotations
@@ -25,6 +32,7 @@ import argparse
 import dataclasses
 import json
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -40,6 +48,14 @@ METRIC = "MLA decode cached-token·heads/s and % of HBM / bf16 tensor-core roofl
 UNIT = "cached-token·heads/s"
 ROW_BYTES = 576 * 2                 # one cached row: c (512) + k_R (64), bf16
 FLOP_PER_ROW_HEAD = 2 * 576 + 2 * 512
+
+# Launches of this library per decode step (checked against the ncu launch
+# list): append 2 (W_DKV + W_KR projection with its in-cluster split-K sum;
+# RMSNorm / RoPE / page write), absorb_q 2 (W_DQ, in-cluster split-K; the fused
+# per-head W_UQ + W_QR + RoPE + W_UK kernel), decode_attn 3 (plan, attention,
+# merge), unabsorb_out 2 (W_UV; W_O with its in-cluster split-K sum).
+LAUNCHES_FULL_STEP = 9
+LAUNCHES_ATTENTION = 3
 
 
 def peaks():
@@ -62,12 +78,25 @@ def workload(name, rank):
     return dataclasses.replace(base, wid=base.wid + 100 * rank)
 
 
-def describe(wl, lens):
+def attention_only(wl) -> bool:
+    return wl.new_tokens == 0
+
+
+def describe(wl):
+    if attention_only(wl):
+        what = "latent attention only (plan + attention + split merge) over the cached rows"
+        rows = f"{wl.prior_min} rows per sequence (the query's own included)"
+    else:
+        what = "full layer step: append + absorb_q (W_DQ) + attention + unabsorb (W_UV, W_O)"
+        rows = f"cached rows {wl.prior_min}..{wl.prior_max} + {wl.new_tokens} new"
     return (f"{wl.name}: batch {wl.batch}/GPU, {wl.n_heads} heads, d_model {wl.d_model}, "
             f"q_lora {wl.d_q}, d_c {wl.d_c}, d_rope {wl.d_rope}, d_nope {wl.d_nope}, d_v {wl.d_v}, "
-            f"cached rows {wl.prior_min}..{wl.prior_max} + {wl.new_tokens} new, "
-            f"{wl.page_size}-row pages{' (shuffled)' if wl.shuffle_pages else ''}; "
-            f"full layer step: append + absorb_q (W_DQ) + attention + unabsorb (W_UV, W_O)")
+            f"{rows}, {wl.page_size}-row pages{' (shuffled)' if wl.shuffle_pages else ''}; {what}")
+
+
+def attended_lengths(wl, prior):
+    """Rows each sequence's query attends to."""
+    return prior if attention_only(wl) else prior + 1
 
 
 def algorithmic(wl, lens):
@@ -76,6 +105,9 @@ def algorithmic(wl, lens):
     rows = int(lens.sum())
     attn_bytes = rows * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 2   # cache + q_lat + z
     attn_flops = rows * H * FLOP_PER_ROW_HEAD
+    if attention_only(wl):
+        return dict(rows=rows, attn_bytes=attn_bytes, attn_flops=attn_flops,
+                    step_bytes=attn_bytes, step_flops=attn_flops, params=0)
     dq = wl.d_q or wl.d_model
     params = (wl.d_c + wl.d_rope) * wl.d_model + (wl.d_q * wl.d_model if wl.d_q else 0) \
         + H * (wl.d_nope + wl.d_rope) * dq + H * wl.d_nope * wl.d_c + H * wl.d_v * wl.d_c \
@@ -87,70 +119,83 @@ def algorithmic(wl, lens):
 
 
 # ---------------------------------------------------------------------------
-# clocks sampled during the timed region
+# clocks sampled during the timed region (read-only NVML queries)
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    """Polls the SM clock, the power draw and the active clock-event reasons of
+    one GPU through NVML every ~0.5 ms on a background thread, so that even a
+    timed region of a few milliseconds holds samples.  Reads only."""
 
-    def __init__(self, gpu_id):
-        self.gpu_id = gpu_id
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("sw_power_cap", 0x4))
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
         self.samples = []
-        self.proc = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20", "-i", str(self.gpu_id)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            pynvml.nvmlInit()
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
             return
-        threading.Thread(target=self._read, daemon=True).start()
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+    def _poll(self):
+        import pynvml
+        while not self._stop.is_set():
+            try:
+                t = time.time()
+                sm = pynvml.nvmlDeviceGetClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+                rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                pw = pynvml.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+            except Exception:
+                return
+            self.samples.append((t, sm, rs, pw))
+            time.sleep(0.0005)
 
     def stop(self):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
 
-    def summary(self, t0, t1):
-        if self.proc is None:
+    def summary(self, windows):
+        """Samples inside the given (t0, t1) wall-clock windows."""
+        if self._thread is None or not self.samples:
             return None
-        inside = [s for t, s in self.samples if t0 <= t <= t1]
-        # a short timed region may hold no sample: then use the ones within 0.25 s of it
-        near = [s for t, s in self.samples if t0 - 0.25 <= t <= t1 + 0.25]
-        used = inside or near or [s for _, s in self.samples]
-        sm, mx, reasons = [], [], set()
-        for s in used:
-            try:
-                sm.append(float(s[1]))
-                mx.append(float(s[2]))
-            except (ValueError, IndexError):
-                continue
-            for name, v in zip(self.NAMES, s[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(used), "samples_in_timed_region": len(inside),
-                "sample_interval_ms": 20}
+        inside = [s for s in self.samples if any(t0 <= s[0] <= t1 for t0, t1 in windows)]
+        used = inside or self.samples
+        reasons = sorted({name for s in used for name, bit in self.REASONS if s[2] & bit})
+        return {"sm_mhz": statistics.median(s[1] for s in used), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "power_w_median": statistics.median(s[3] for s in used),
+                "samples_in_timed_region": len(inside), "source": "nvml, ~0.5 ms polling"}
 
 
 # ---------------------------------------------------------------------------
-# our implementation
+# ranks
 # ---------------------------------------------------------------------------
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(nproc, argv):
+    """Re-runs this script under torch.distributed.run with one rank per GPU
+    (used when --gpus N > 1 is given outside a torchrun launch)."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={nproc}", "--master-addr", "127.0.0.1",
+           "--master-port", str(_free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
 
 def setup_dist(args, backend="nccl"):
     """Process group from the torchrun environment (one rank per GPU; ``gloo`` for
@@ -180,30 +225,55 @@ def max_over_ranks(values, world, device):
     return t.tolist()
 
 
-def cpu_baseline_sample(wl, W, pc, h, lens, budget_s=20.0):
-    """The oracle's whole decode step (un-absorbed form) on a bounded sample."""
+# ---------------------------------------------------------------------------
+# the oracle's CPU time (baseline only; never on the timed path)
+# ---------------------------------------------------------------------------
+
+def _threads():
+    try:
+        import threadpoolctl
+        return max((p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()), default=1)
+    except Exception:
+        return 1
+
+
+def _oracle_dims(wl):
     import oracle
-    od = oracle.Dims(n_heads=wl.n_heads, d_c=wl.d_c, d_rope=wl.d_rope, d_nope=wl.d_nope,
-                     d_v=wl.d_v, rope_base=wl.rope_base, rms_eps=wl.rms_eps,
-                     rope_layout=wl.rope_layout)
-    # calibrate on a short prefix of sequence 0, then size the sample to the budget
+    return oracle.Dims(n_heads=wl.n_heads, d_c=wl.d_c, d_rope=wl.d_rope, d_nope=wl.d_nope,
+                       d_v=wl.d_v, rope_base=wl.rope_base, rms_eps=wl.rms_eps,
+                       rope_layout=wl.rope_layout)
+
+
+def _oracle_unit(wl, W, pc, h, q):
+    """f(b, n): the oracle's work for sequence b over its first n attended rows
+    (a whole un-absorbed decode step, or the latent attention alone)."""
+    import oracle
+    od = _oracle_dims(wl)
+    if attention_only(wl):
+        return lambda b, n: oracle.attend_latent(q[b], pc.rows_f32(b, n), od)
+    return lambda b, n: oracle.decode_step(h[b:b + 1], [pc.rows_f32(b, n - 1)], W, od)
+
+
+def cpu_baseline_sample(wl, W, pc, h, q, lens, budget_s=20.0):
+    """The oracle on a bounded sample of the workload: one sequence over a prefix."""
+    f = _oracle_unit(wl, W, pc, h, q)
     t = time.perf_counter()
-    oracle.decode_step(h[:1], [pc.rows_f32(0, 63)], W, od)
+    f(0, 64)
     per_row = (time.perf_counter() - t) / 64
     n = int(min(lens[0], max(64, budget_s / max(per_row, 1e-9))))
     t = time.perf_counter()
-    oracle.decode_step(h[:1], [pc.rows_f32(0, n - 1)], W, od)
+    f(0, n)
     dt = time.perf_counter() - t
-    try:
-        import threadpoolctl
-        threads = max((p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()), default=1)
-    except Exception:
-        threads = 1
-    return {"value": n * wl.n_heads / dt, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": f"sequence 0 of {wl.name}, first {n} cached rows (new token included), "
-                      f"all {wl.n_heads} heads, one whole un-absorbed fp64 decode step "
-                      f"({dt:.1f} s)", "host_cpus": os.cpu_count()}
+    form = ("latent attention" if attention_only(wl) else "whole un-absorbed decode step")
+    return {"value": n * wl.n_heads / dt, "unit": UNIT, "cores": int(_threads()), "kind": "oracle",
+            "sample": f"sequence 0 of {wl.name}, first {n} attended rows (new token included), "
+                      f"all {wl.n_heads} heads, one fp64 {form} ({dt:.1f} s)",
+            "host_cpus": os.cpu_count()}
 
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
 
 def run_mine(args):
     import torch
@@ -215,94 +285,145 @@ def run_mine(args):
     torch.cuda.set_device(local)
     build.build()
     wl = workload(args.workload, rank)
-    assert wl.new_tokens == 1, "the bench runs whole decode steps"
-    W = synth.make_weights(wl)
+    attn_only = attention_only(wl)
     prior = synth.make_prior_lengths(wl)
+    lens = attended_lengths(wl, prior)
     pc = synth.make_paged_cache(wl, prior)
-    h = synth.make_hidden(wl)
-    lens = prior + 1
+    W = None if attn_only else synth.make_weights(wl)
+    h = None if attn_only else synth.make_hidden(wl)
+    q = synth.make_q_lat(wl) if attn_only else None
     dims = L.Dims(wl.n_heads, wl.d_c, wl.d_rope, wl.d_nope, wl.d_v, wl.page_size, L.MLA_BF16,
                   wl.rope_layout, wl.rope_base, wl.rms_eps)
     dev = torch.device("cuda", local)
-    Wd = {k: (None if v is None else torch.from_numpy(v).to(dev).to(torch.bfloat16))
-          for k, v in W.items()}
+    bf = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
     pool = torch.from_numpy(pc.pool.view(np.int16)).to(dev).view(torch.bfloat16)
     cache = L.PagedCache(pool, torch.from_numpy(pc.block_table).to(dev),
                          torch.from_numpy(lens.astype(np.int32)).to(dev))
-    hd = torch.from_numpy(h).to(dev).to(torch.bfloat16)
-    pos = torch.from_numpy(prior.astype(np.int32)).to(dev)
-    layer = DecodeLayer(dims, Wd, wl.batch, args.num_splits, device=dev)
     stream = torch.cuda.current_stream()
+    if attn_only:
+        # attention alone: q_lat in, z / lse out
+        q_dev = bf(q)
+        n_ws = L.mla_workspace_size(dims, wl.batch, 64, 0, args.num_splits)
+        ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+        L.mla_workspace_init(ws)
+        z = torch.empty(wl.batch, wl.n_heads, wl.d_c, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(wl.batch, wl.n_heads, dtype=torch.float32, device=dev)
 
-    def step():
-        layer.step(cache, hd, pos)
+        def step(e=None):
+            if e:
+                e[4].record(stream)
+            L.mla_decode_attn(dims, cache, q_dev, z, lse, args.num_splits, ws, stream)
+            if e:
+                e[5].record(stream)
+
+        def device_error():
+            return L.mla_get_device_error(ws)
+
+        inputs, output = [q_dev], z
+        launches = LAUNCHES_ATTENTION
+    else:
+        Wd = {k: (None if v is None else bf(v)) for k, v in W.items()}
+        hd = bf(h)
+        pos = torch.from_numpy(prior.astype(np.int32)).to(dev)
+        layer = DecodeLayer(dims, Wd, wl.batch, args.num_splits, device=dev)
+
+        def step(e=None):
+            layer.step(cache, hd, pos, stream, e)
+
+        device_error = layer.device_error
+        inputs, output = [hd, pos, cache.seq_lens], layer.out
+        launches = LAUNCHES_FULL_STEP
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    st = layer.device_error()
+    st = device_error()
     if st != 0:
         raise RuntimeError(f"device error {L.STATUS.get(st)} during warm-up")
 
-    # per-call events inside the timed region: the append on the layer's side
-    # stream, the other calls on the main stream (see DecodeLayer.step)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    # one step captured as a CUDA graph (the same launches, replayed)
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(device=dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        stream_saved = stream
+        stream = cap
+        with torch.cuda.graph(graph, stream=cap):
+            step()
+        stream = stream_saved
+    stream.wait_stream(cap)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
 
-    def timed_step(e):
-        layer.step(cache, hd, pos, stream, e)
-
-    gpu_id = torch.cuda.get_device_properties(dev).uuid
-    gpu_id = f"GPU-{gpu_id}" if not str(gpu_id).startswith("GPU-") else gpu_id
-    clocks = ClockSampler(gpu_id) if rank == 0 else None
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}") if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.5)
+        time.sleep(0.2)
+    windows = []
+
+    # ---- timed region: K steps, barrier + synchronize on both sides
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
-    for k in range(args.steps):
-        timed_step(ev[k])
+    for _ in range(args.steps):
+        graph.replay()
     end.record(stream)
     torch.cuda.synchronize()
-    t_wall1 = time.time()
+    windows.append((t_wall0, time.time()))
     if world > 1:
         torch.distributed.barrier()
     elapsed = start.elapsed_time(end)  # ms
-    per_call = np.array([[e[0].elapsed_time(e[1]), e[2].elapsed_time(e[3]),
-                          e[4].elapsed_time(e[5]), e[5].elapsed_time(e[6])] for e in ev])
-    st = layer.device_error()
+    st = device_error()
     if st != 0:
         raise RuntimeError(f"device error {L.STATUS.get(st)} in the timed region")
-    if clocks:
-        clocks.stop()
 
-    # end-to-end through the public API with host buffers: pinned h2d of the
-    # step's inputs and d2h of its output inside the timed region
-    h_host = hd.cpu().pin_memory()
-    pos_host = pos.cpu().pin_memory()
-    lens_host = cache.seq_lens.cpu().pin_memory()
-    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-    for _ in range(max(3, args.warmup // 4)):
-        hd.copy_(h_host, non_blocking=True)
-        step()
-        out_host.copy_(layer.out, non_blocking=True)
+    # ---- per-call breakdown (eager, events around each call on its own stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_b0 = time.time()
+    for k in range(args.steps):
+        step(ev[k])
+    torch.cuda.synchronize()
+    windows.append((t_b0, time.time()))
+    if attn_only:
+        per_call = np.array([[0.0, 0.0, e[4].elapsed_time(e[5]), 0.0] for e in ev])
+    else:
+        per_call = np.array([[e[0].elapsed_time(e[1]), e[2].elapsed_time(e[3]),
+                              e[4].elapsed_time(e[5]), e[5].elapsed_time(e[6])] for e in ev])
+
+    # ---- end-to-end through the Python API with host buffers: pinned h2d of the
+    # step's inputs and d2h of its output inside the timed region, eager calls
+    host_in = [t.cpu().pin_memory() for t in inputs]
+    out_host = torch.empty(output.shape, dtype=output.dtype).pin_memory()
+
+    def e2e_step():
+        for d, hbuf in zip(inputs, host_in):
+            d.copy_(hbuf, non_blocking=True)
+        step()
+        out_host.copy_(output, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        hd.copy_(h_host, non_blocking=True)
-        pos.copy_(pos_host, non_blocking=True)
-        cache.seq_lens.copy_(lens_host, non_blocking=True)
-        step()
-        out_host.copy_(layer.out, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    if clocks:
+        clocks.stop()
+    st = device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {L.STATUS.get(st)} in the end-to-end pass")
 
     elapsed, e2e_ms, attn_ms_total = max_over_ranks([elapsed, e2e_ms, per_call[:, 2].sum()],
                                                     world, dev)
@@ -319,48 +440,47 @@ def run_mine(args):
         achieved, peak, unit = alg["attn_bytes"] / (attn_ms / 1e3) / 1e9, hbm, "GB/s"
     else:
         achieved, peak, unit = alg["attn_flops"] / (attn_ms / 1e3) / 1e12, tf, "TFLOP/s"
-    traffic = stored_traffic(wl.name.split("+")[0])
     step_t = max(alg["step_bytes"] / (hbm * 1e9), alg["step_flops"] / (tf * 1e12))
-    h2d = (hd.numel() * hd.element_size() + pos.numel() * 4 + cache.seq_lens.numel() * 4)
-    d2h = layer.out.numel() * layer.out.element_size()
+    h2d = sum(t.numel() * t.element_size() for t in inputs)
+    d2h = output.numel() * output.element_size()
+    l2 = ("no flush: per-step inputs (cache %.0f MB%s) exceed the 126 MB L2"
+          % (alg["rows"] * ROW_BYTES / 1e6,
+             "" if attn_only else " + weights %.0f MB" % (2 * alg["params"] / 1e6)))
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(wl, lens), "batch_per_gpu": wl.batch,
+        "config": {"workload": describe(wl), "batch_per_gpu": wl.batch,
                    "global_batch": wl.batch * world, "cached_rows_per_step": alg["rows"],
                    "parallelism": f"dp{world} (sequences sharded, no collective)",
-                   "l2": "no flush: per-step inputs (cache %.0f MB + weights %.0f MB) exceed the "
-                         "126 MB L2" % (alg["rows"] * ROW_BYTES / 1e6, 2 * alg["params"] / 1e6),
-                   "num_splits": args.num_splits},
+                   "l2": l2, "num_splits": args.num_splits,
+                   "timed": "one captured CUDA graph of the step, replayed K times"},
         "roofline": {"kernel": "mla_decode_attn (plan + attention + split merge)",
                      "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": traffic, "peak_source": src,
+                     "frac": achieved / peak,
+                     "traffic": stored_traffic(wl.name),
+                     "peak_source": src,
                      "algorithmic_bytes": alg["attn_bytes"], "algorithmic_flops": alg["attn_flops"],
-                     "ms_per_launch": attn_ms},
+                     "ms_per_launch": attn_ms,
+                     "timing": "CUDA events around each call in an eager pass of K steps"},
         "step_roofline": {"bytes": alg["step_bytes"], "flops": alg["step_flops"],
                           "roofline_ms": step_t * 1e3, "frac": step_t * 1e3 / ms_step},
         "breakdown_ms": dict(zip(["cache_append", "absorb_q", "decode_attn", "unabsorb_out"],
                                  [float(x) for x in per_call.mean(0)])),
         "e2e": {"value": alg["rows"] * wl.n_heads * world / (e2e_ms / args.steps / 1e3),
                 "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-                "ms_per_step": e2e_ms / args.steps},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+                "ms_per_step": e2e_ms / args.steps,
+                "how": "eager API calls per step, pinned host copies in and out on the stream"},
+        "gpu_launches": launches * args.steps,
     }
     if rank == 0:
-        res["clocks"] = clocks.summary(t_wall0, t_wall1) if clocks else None
+        res["clocks"] = clocks.summary(windows) if clocks else None
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline_sample(wl, W, pc, h, lens)
+            res["cpu_baseline"] = cpu_baseline_sample(wl, W, pc, h, q, lens)
         print(json.dumps(res), flush=True)
+    del graph
     if world > 1:
         torch.distributed.destroy_process_group()
-
-
-# Launches of this library per decode step (checked against the ncu launch list):
-# append 2 (W_DKV+W_KR projection, RMSNorm/RoPE/page write), absorb_q 5 (W_DQ,
-# its split-K reduce, W_UQ+W_QR, W_UK, RoPE), decode_attn 3 (plan, attention,
-# merge), unabsorb_out 3 (W_UV, W_O, its split-K reduce).
-LAUNCHES_PER_STEP = 13
 
 
 ATTN_SOURCES = ("attn_sm100.cu", "kernels_simt.cu", "ptx.cuh", "common.cuh", "kernels.h", "sm100.h")
@@ -398,52 +518,60 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import oracle
     from mla_latent_kv_45_b200 import synth
     wl = workload(args.workload, 0)
-    W = synth.make_weights(wl)
     prior = synth.make_prior_lengths(wl)
+    lens = attended_lengths(wl, prior)
     pc = synth.make_paged_cache(wl, prior)
-    h = synth.make_hidden(wl)
-    od = oracle.Dims(n_heads=wl.n_heads, d_c=wl.d_c, d_rope=wl.d_rope, d_nope=wl.d_nope,
-                     d_v=wl.d_v, rope_base=wl.rope_base, rms_eps=wl.rms_eps,
-                     rope_layout=wl.rope_layout)
+    attn_only = attention_only(wl)
+    W = None if attn_only else synth.make_weights(wl)
+    h = None if attn_only else synth.make_hidden(wl)
+    q = synth.make_q_lat(wl) if attn_only else None
+    f = _oracle_unit(wl, W, pc, h, q)
     # size each step's sample so the whole run stays within ~2 minutes
     t = time.perf_counter()
-    oracle.decode_step(h[:1], [pc.rows_f32(0, 63)], W, od)
+    f(0, 64)
     per_row = (time.perf_counter() - t) / 64
     budget = 120.0 / max(1, args.steps + args.warmup)
-    n = int(min(prior[0] + 1, max(16, budget / max(per_row, 1e-9))))
-    rows = [pc.rows_f32(b % wl.batch, n - 1) for b in range(wl.batch)]
-
-    def one(k):
-        b = k % wl.batch
-        oracle.decode_step(h[b:b + 1], [rows[b]], W, od)
+    n = int(min(lens.min(), max(16, budget / max(per_row, 1e-9))))
 
     for k in range(args.warmup):
-        one(k)
+        f(k % wl.batch, n)
     t0 = time.perf_counter()
     for k in range(args.steps):
-        one(k)
+        f(k % wl.batch, n)
     dt = time.perf_counter() - t0
     value = n * wl.n_heads * args.steps / dt
-    try:
-        import threadpoolctl
-        threads = max((p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()), default=1)
-    except Exception:
-        threads = 1
+    form = "latent attention" if attn_only else "whole un-absorbed fp64 decode step"
     sample = (f"each step: one sequence of {wl.name} (cycling over its {wl.batch}), first {n} "
-              f"cached rows incl. the new token, all {wl.n_heads} heads, whole un-absorbed fp64 "
-              f"decode step")
+              f"attended rows incl. the new token, all {wl.n_heads} heads, {form}")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": describe(wl, prior + 1)},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+        "data": "synthetic", "config": {"workload": describe(wl)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": int(_threads()), "kind": "oracle",
                          "sample": sample, "host_cpus": os.cpu_count()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# multi-rank plumbing check without a GPU
+# ---------------------------------------------------------------------------
+
+def run_rank_check(args):
+    """Each rank reports a rank-dependent timing through the same max-over-ranks
+    reduction the bench uses (gloo, no GPU); rank 0 prints one line."""
+    rank, world, _ = setup_dist(args, backend="gloo")
+    wl = workload(args.workload, rank)
+    got = max_over_ranks([1.0 + rank, float(wl.wid)], world, "cpu")
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "max_ms": got[0], "max_wid": got[1]}), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def main():
@@ -455,10 +583,16 @@ def main():
     ap.add_argument("--workload", default="v2_batch64")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rank-check", action="store_true",
+                    help="run only the multi-rank plumbing on CPU (gloo), no GPU work")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
+    if args.rank_check:
+        run_rank_check(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_mine(args)

@@ -138,8 +138,10 @@ mla_status mla_cache_append(const mla_dims *dims, const mla_paged_cache *cache, 
  *   q_lat[b][i] = [W_UK,i^T q_C,i ; q_R,i]   (d_c + d_rope values).
  * x: [batch][d_in]; W_DQ: [d_q][d_in] or NULL; W_UQ: [n_heads*d_nope][d_q];
  * W_QR: [n_heads*d_rope][d_q]; W_UK: [n_heads*d_nope][d_c];
- * q_lat: [batch][n_heads][d_c + d_rope] (output).  Intermediates c_Q and q_C
- * stay in fp32 inside the workspace. */
+ * q_lat: [batch][n_heads][d_c + d_rope] (output).  Intermediates live in the
+ * workspace: with MLA_BF16, c_Q and q_C are stored as bf16 (as a bf16 model
+ * stores activations) and q_R stays fp32 until it is rotated and rounded once
+ * into q_lat; with MLA_FP32 all of them are fp32. */
 mla_status mla_absorb_q(const mla_dims *dims, int batch, int d_in, const void *x,
                         const void *W_DQ, int d_q, const void *W_UQ, const void *W_QR,
                         const void *W_UK, const int32_t *positions, void *q_lat, void *ws,
@@ -159,6 +161,33 @@ mla_status mla_absorb_q(const mla_dims *dims, int batch, int d_in, const void *x
 mla_status mla_decode_attn(const mla_dims *dims, const mla_paged_cache *cache, int batch,
                            const void *q_lat, void *z, float *lse, int num_splits, void *ws,
                            size_t ws_bytes, mla_stream_t stream);
+
+/* Partial softmax of decode attention, for a sequence whose cached rows are
+ * split across devices (each device holds some of its pages and attends over
+ * them; the partials are then gathered and merged with mla_merge_partials).
+ * Same arguments and rows as mla_decode_attn, but instead of z / lse it writes,
+ * for each b and head i over the rows this cache holds:
+ *   m[b][i] = max_s logit_s (natural log units),  l[b][i] = sum_s e^(logit_s - m),
+ *   O[b][i] = sum_s e^(logit_s - m) c_s            (fp32, not normalised),
+ * with logit_s = scale * q_lat[b][i] . row_s.  z_i = O_i / l_i over these rows
+ * alone; several shares merge as in mla_merge_partials.  This is the standard
+ * rewriting of one softmax as a weighted merge of partial softmaxes; the pages
+ * describe no split.  O: [batch][n_heads][d_c] (16-byte aligned); m, l:
+ * [batch][n_heads].  A sequence with seq_lens[b] == 0 (no rows on this device)
+ * is an empty share: O = 0, m = -inf, l = 0, and no error is recorded. */
+mla_status mla_decode_attn_partial(const mla_dims *dims, const mla_paged_cache *cache, int batch,
+                                   const void *q_lat, float *O, float *m, float *l, int num_splits,
+                                   void *ws, size_t ws_bytes, mla_stream_t stream);
+
+/* Merges n_parts partial softmaxes (e.g. one per device, gathered):
+ *   M = max_j m_j,  w_j = e^(m_j - M),  z = sum_j w_j O_j / sum_j w_j l_j,
+ *   lse = M + log(sum_j w_j l_j)   (parts summed in increasing j).
+ * O: [n_parts][batch][n_heads][d_c] fp32; m, l: [n_parts][batch][n_heads];
+ * z: [batch][n_heads][d_c] of dims->dtype; lse: [batch][n_heads] or NULL.
+ * A row whose parts are all empty (m = -inf) gets z = 0, lse = -inf. */
+mla_status mla_merge_partials(const mla_dims *dims, int batch, int n_parts, const float *O,
+                              const float *m, const float *l, void *z, float *lse,
+                              mla_stream_t stream);
 
 /* Value up-projection after latent aggregation ("从零理解 MLA", 矩阵吸收: value
  * side, o_{t,i} = W_i^UV z_{t,i}; absorbed_step: o, then w_o).  For each b:
@@ -181,21 +210,40 @@ mla_status mla_unabsorb_out(const mla_dims *dims, int batch, const void *z, cons
  * the library until the process exits.  num_splits = 0 picks the most
  * partitions that fit (at most one per pair of SMs); a batch or num_splits
  * whose scratch would exceed 16 MiB returns MLA_ERR_WORKSPACE before any work
- * is enqueued (for the bf16 sizes: about 60 partitions at small batch).
+ * is enqueued (for the bf16 sizes: at most 30 partitions, i.e. 60 of the SMs).
  * The first call on a device looks up the array's device address for that
  * device; make it before any stream capture.  Calls share the array: calls
  * whose work overlaps on the GPU race and must be serialised by the caller.
  * Device-side range errors zero the affected sequence (z = 0, lse = -inf) as in
- * mla_decode_attn; the error word itself is cleared at the start of each call
- * and is not readable by the caller. */
+ * mla_decode_attn.  The array's error word is cleared at the start of each call
+ * and read with mla_noalloc_get_device_error; after MLA_ERR_TIMEOUT (a bounded
+ * wait inside the kernels gave up) z and lse of that call are not valid. */
 mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_paged_cache *cache, int batch,
                                    const void *q_lat, void *z, float *lse, int num_splits,
                                    mla_stream_t stream);
+
+/* The device status of the most recent mla_decode_attn_noalloc call on the
+ * current device: waits for `stream` (the stream of that call), then reads and
+ * clears the error word of the library's fixed scratch array.  Returns MLA_OK,
+ * MLA_ERR_DEVICE_RANGE or MLA_ERR_TIMEOUT (MLA_ERR_CUDA if the stream failed).
+ * Like the call it reports on, it allocates nothing and synchronises only. */
+mla_status mla_noalloc_get_device_error(mla_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the workspace's device error word.
  * Returns MLA_OK, MLA_ERR_DEVICE_RANGE or MLA_ERR_TIMEOUT (or MLA_ERR_CUDA if
  * the stream itself failed).  This is the only call that synchronises. */
 mla_status mla_get_device_error(void *ws, mla_stream_t stream);
+
+/* Test hook, not for production use: exercises the bounded waits.  With
+ * enable != 0, every later mla_absorb_q (MLA_BF16) call bounds each of its
+ * kernel's internal waits by wait_limit_us microseconds (instead of 2 s) and
+ * makes one epilogue warp of the per-head absorption kernel withhold its arrive
+ * on the barrier that hands the q_C tile to the W_UK products; that wait then
+ * runs out, the kernel records MLA_ERR_TIMEOUT in the workspace error word,
+ * drains the loads and MMAs it issued and exits (q_lat is not valid).
+ * enable = 0 restores normal operation.  Process-wide; not thread-safe with
+ * concurrent mla_absorb_q calls.  No page describes this; it exists for tests. */
+mla_status mla_debug_absorb_timeout(int enable, unsigned wait_limit_us);
 
 /* Static, NUL-terminated description of a status code. */
 const char *mla_status_string(mla_status status);

@@ -26,8 +26,10 @@ STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
           6: "MLA_ERR_DEVICE_RANGE", 7: "MLA_ERR_TIMEOUT"}
 
 EXPORTS = ("mla_workspace_size", "mla_workspace_init", "mla_cache_append", "mla_absorb_q",
-           "mla_decode_attn", "mla_decode_attn_noalloc", "mla_unabsorb_out",
-           "mla_get_device_error", "mla_status_string")
+           "mla_decode_attn", "mla_decode_attn_partial", "mla_merge_partials",
+           "mla_decode_attn_noalloc", "mla_unabsorb_out",
+           "mla_noalloc_get_device_error", "mla_get_device_error", "mla_debug_absorb_timeout",
+           "mla_status_string")
 
 
 class MlaError(RuntimeError):
@@ -107,9 +109,13 @@ def lib() -> ctypes.CDLL:
         L.mla_cache_append.argtypes = [pd, pc, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.mla_absorb_q.argtypes = [pd, i, i, vp, vp, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.mla_decode_attn.argtypes = [pd, pc, i, vp, vp, vp, i, vp, sz, vp]
+        L.mla_decode_attn_partial.argtypes = [pd, pc, i, vp, vp, vp, vp, i, vp, sz, vp]
+        L.mla_merge_partials.argtypes = [pd, i, i, vp, vp, vp, vp, vp, vp]
         L.mla_decode_attn_noalloc.argtypes = [pd, pc, i, vp, vp, vp, i, vp]
         L.mla_unabsorb_out.argtypes = [pd, i, vp, vp, vp, i, vp, vp, sz, vp]
         L.mla_get_device_error.argtypes = [vp, vp]
+        L.mla_noalloc_get_device_error.argtypes = [vp]
+        L.mla_debug_absorb_timeout.argtypes = [i, ctypes.c_uint]
         L.mla_status_string.argtypes = [i]
         L.mla_status_string.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -174,6 +180,23 @@ def mla_decode_attn(dims: Dims, cache: PagedCache, q_lat, z, lse=None, num_split
         _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
+def mla_decode_attn_partial(dims: Dims, cache: PagedCache, q_lat, O, m, l, num_splits: int = 0,
+                            ws: torch.Tensor = None, stream=None):
+    """Unnormalised partial softmax (O, m, l) over the rows this cache holds."""
+    d, c = dims.c(), cache.c()
+    _ok("mla_decode_attn_partial", lib().mla_decode_attn_partial(
+        ctypes.byref(d), ctypes.byref(c), q_lat.shape[0], _p(q_lat), _p(O), _p(m), _p(l),
+        num_splits, _p(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def mla_merge_partials(dims: Dims, O, m, l, z, lse=None, stream=None):
+    """z (and lse) from partials stacked as O [n, B, H, d_c], m and l [n, B, H]."""
+    d = dims.c()
+    _ok("mla_merge_partials", lib().mla_merge_partials(
+        ctypes.byref(d), O.shape[1], O.shape[0], _p(O), _p(m), _p(l), _p(z), _p(lse),
+        _stream(stream)))
+
+
 def mla_decode_attn_noalloc(dims: Dims, cache: PagedCache, q_lat, z, lse=None,
                             num_splits: int = 0, stream=None):
     """Decode attention with the library's fixed internal scratch (no workspace)."""
@@ -189,6 +212,17 @@ def mla_unabsorb_out(dims: Dims, z, W_UV, W_O, out, ws: torch.Tensor, stream=Non
     _ok("mla_unabsorb_out", lib().mla_unabsorb_out(
         ctypes.byref(d), z.shape[0], _p(z), _p(W_UV), _p(W_O), d_model, _p(out), _p(ws),
         ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def mla_noalloc_get_device_error(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status of the last
+    allocation-free decode-attention call on the current device."""
+    return int(lib().mla_noalloc_get_device_error(_stream(stream)))
+
+
+def mla_debug_absorb_timeout(enable: bool, wait_limit_us: int = 0):
+    """Test hook: make the absorption kernel's q_C hand-off wait run out (see mla.h)."""
+    _ok("mla_debug_absorb_timeout", lib().mla_debug_absorb_timeout(int(enable), wait_limit_us))
 
 
 def mla_get_device_error(ws: torch.Tensor, stream=None) -> int:

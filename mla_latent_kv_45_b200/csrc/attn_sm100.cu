@@ -47,6 +47,7 @@
 //    and exits.  No TMA multicast is used.
 #include <cuda.h>
 
+#include "api_checks.h"
 #include "ptx.cuh"
 #include "sm100.h"
 
@@ -55,6 +56,13 @@ namespace sm100 {
 namespace {
 
 using namespace ptx;
+
+#ifndef MLA_ATTN_PREFETCH
+#define MLA_ATTN_PREFETCH 0   // steps of L2 prefetch ahead of the row ring (0 = none)
+#endif
+#ifndef MLA_ATTN_PV_FIRST
+#define MLA_ATTN_PV_FIRST 0   // 1: score MMAs of step i + 2 wait until P.V(i) is issued
+#endif
 
 constexpr int kHeads = 128;
 constexpr int kRow = 576;        // cached values per row
@@ -122,6 +130,7 @@ struct Bars {
   uint64_t drain_s, drain_pv;
   uint32_t tmem_base;
   volatile int abort;
+  volatile int pv_issued;     // even CTA: steps whose P.V MMAs have been issued
 };
 
 struct Ctx {
@@ -145,6 +154,24 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, uint64_t *bar, uint32_t p
     }
   }
 }
+
+#if MLA_ATTN_PV_FIRST
+// Bounded wait until a counter in this CTA's shared memory reaches `target`.
+__device__ __forceinline__ bool wait_count(const Ctx &c, volatile int *counter, int target) {
+  if (*counter >= target) return true;
+  const uint64_t t0 = globaltimer();
+  while (*counter < target) {
+    if (c.bars->abort) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      set_error(c.err, kErrTimeout);
+      c.bars->abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
+#endif
 
 // Waits (bounded, ignoring the abort flag) for asynchronous work this CTA issued.
 __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
@@ -293,6 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&bars->drain_s, 1);
     mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
+    bars->pv_issued = 0;
     fence_mbar_init();
   }
   if (warp == kWarpLoad && lane == 0) {
@@ -321,7 +349,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int nk = 0;
       bool ok = true;
+#if MLA_ATTN_PREFETCH > 0
+      // this CTA's pages MLA_ATTN_PREFETCH steps ahead are brought into L2, so the
+      // row loads of the ring hit L2 instead of waiting a full DRAM latency
+      StepCursor ahead = cur;
+      for (int d = 0; d < MLA_ATTN_PREFETCH && ahead.valid; ++d) {
+        for (int sp = 0; sp < 2; ++sp) {
+          const int j = 2 * (int)rank + sp;
+          if (j < ahead.npages()) {
+            const int page = ahead.page(a, j);
+            if (page >= 0 && page < a.num_pages)
+              prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRow * 2,
+                          kPage * kRow * 2);
+          }
+        }
+        ahead.advance(a);
+      }
+#endif
       for (; cur.valid && ok; cur.advance(a)) {
+#if MLA_ATTN_PREFETCH > 0
+        if (ahead.valid) {
+          for (int sp = 0; sp < 2; ++sp) {
+            const int j = 2 * (int)rank + sp;
+            if (j < ahead.npages()) {
+              const int page = ahead.page(a, j);
+              if (page >= 0 && page < a.num_pages)
+                prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRow * 2,
+                            kPage * kRow * 2);
+            }
+          }
+          ahead.advance(a);
+        }
+#endif
         const int np = cur.npages();
         int pages[2];
         for (int sp = 0; sp < 2; ++sp) {
@@ -429,6 +488,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int sb = step & 1;
         // score buffer sb was last read by the softmax of step - 2
         if (step >= 2 && !wait_bar(ctx, &bars->s_free[sb], ((step >> 1) - 1) & 1)) break;
+#if MLA_ATTN_PV_FIRST
+        // keep P.V(step - 2) ahead of these score MMAs on the tensor pipe
+        if (step >= 2 && !wait_count(ctx, &bars->pv_issued, step - 1)) break;
+#endif
         const uint32_t sd = tmem + kTmemS + 128 * sb;
         for (int c = 0; c < 9; ++c, ++nk) {
           const int slot = nk % kKSlots;
@@ -489,6 +552,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         umma_commit_pair(&bars->pv_done, kBoth);
+#if MLA_ATTN_PV_FIRST
+        bars->pv_issued = step + 1;
+#endif
       }
       umma_commit_pair(&bars->drain_pv, 1);
       drain_bar(&bars->drain_pv, 0);
@@ -648,20 +714,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int pbase = a.part_base[b];
       const bool whole = pbase < 0;
       const int slot_p = whole ? 0 : pbase + (part - tc.seg.s0 / hdr.quota);
+      // a whole sequence writes z (normalised), or, when the caller asked for the
+      // partial softmax, its unnormalised (O, m, l); a piece of a split sequence
+      // writes its partial into the workspace slot the merge reads
+      const bool to_z = whole && !a.pout_O;
+      float *pm = whole ? a.pout_m + (long)b * kHeads : a.part_m + (long)slot_p * kHeads;
+      float *pl = whole ? a.pout_l + (long)b * kHeads : a.part_l + (long)slot_p * kHeads;
+      float *pO = whole ? a.pout_O + (long)b * kHeads * kDc : a.part_O + (long)slot_p * kHeads * kDc;
       if (rank == 0 && quad == 0) {
         const float ln2 = 0.6931471805599453f;
         const int h0 = 64 * g + 2 * lane;
         const long ri = (long)b * kHeads + h0;
-        if (whole) {
+        if (to_z) {
           if (a.lse) {
             a.lse[ri] = (m0 + __log2f(f0)) * ln2;
             a.lse[ri + 1] = (m1 + __log2f(f1)) * ln2;
           }
         } else {
-          a.part_m[(long)slot_p * kHeads + h0] = m0 * ln2;
-          a.part_m[(long)slot_p * kHeads + h0 + 1] = m1 * ln2;
-          a.part_l[(long)slot_p * kHeads + h0] = f0;
-          a.part_l[(long)slot_p * kHeads + h0 + 1] = f1;
+          pm[h0] = m0 * ln2;
+          pm[h0 + 1] = m1 * ln2;
+          pl[h0] = f0;
+          pl[h0 + 1] = f1;
         }
       }
       ok = ok && wait_bar(ctx, &bars->pv_done, i & 1);
@@ -673,13 +746,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float ov[32];
         tmem_ld32f(ob + c, ov);
         tmem_wait_ld();
-        if (whole) {
+        if (to_z) {
           __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + (long)b * kHeads * kDc + col;
 #pragma unroll
           for (int kk = 0; kk < 32; ++kk)
             z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] / lsum[c + kk]);
         } else {
-          float *o = a.part_O + (long)slot_p * kHeads * kDc + col;
+          float *o = pO + col;
 #pragma unroll
           for (int kk = 0; kk < 32; ++kk) o[(long)(c + kk) * kDc] = ov[kk];
         }
@@ -739,13 +812,12 @@ bool make_map(CUtensorMap *m, const void *base, long rows, int box_cols, int box
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static api::PerDeviceOnce smem_attr;
+  cudaError_t e = smem_attr.run([] {
+    return cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
   CUtensorMap tm_rows, tm_q;
   const long pool_rows = (long)a.num_pages * kPage;
   const long q_rows = (long)a.batch * kHeads;

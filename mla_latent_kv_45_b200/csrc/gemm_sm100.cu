@@ -22,6 +22,7 @@
 // warps 2-5 epilogue.  Every wait is bounded (globaltimer).
 #include <cuda.h>
 
+#include "api_checks.h"
 #include "ptx.cuh"
 #include "sm100.h"
 #include "gemm_sm100.h"
@@ -66,10 +67,18 @@ __device__ __forceinline__ Item decode_item(const GemmLaunch &g, int item) {
   it.pi = (g.nprob > 1 && item >= g.p[1].item_begin) ? 1 : 0;
   const GemmProblem &P = g.p[it.pi];
   int t = item - P.item_begin;
-  it.m0 = (t % P.m_tiles) * 128;
-  t /= P.m_tiles;
-  it.split = t % P.splits;
-  it.head = t / P.splits;
+  if (g.cluster) {
+    // split fastest: the splits of one tile are the consecutive CTAs of a cluster
+    it.split = t % P.splits;
+    t /= P.splits;
+    it.m0 = (t % P.m_tiles) * 128;
+    it.head = t / P.m_tiles;
+  } else {
+    it.m0 = (t % P.m_tiles) * 128;
+    t /= P.m_tiles;
+    it.split = t % P.splits;
+    it.head = t / P.splits;
+  }
   it.kc0 = it.split * P.chunks_per_split;
   it.nk = min(g.k_chunks, it.kc0 + P.chunks_per_split) - it.kc0;
   return it;
@@ -177,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const GemmProblem &P = g.p[it.pi];
         const uint32_t idesc = idesc_bf16(128, g.n_pad, P.a_mn, 0);
         const int buf = li & 1;
-        const uint32_t acc = tmem + buf * g.n_pad;
+        const uint32_t acc = tmem + buf * g.n_cols;
         if (li >= 2 && !gwait(bars, g.err, &bars->acc_free[buf], ((li >> 1) - 1) & 1)) break;
         tc_fence_after();
         for (int i = 0; i < it.nk; ++i, ++c) {
@@ -210,12 +219,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int buf = li & 1;
       if (!gwait(bars, g.err, &bars->acc_full[buf], (li >> 1) & 1)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + buf * g.n_pad + (static_cast<uint32_t>(quad * 32) << 16);
+      const uint32_t taddr = tmem + buf * g.n_cols + (static_cast<uint32_t>(quad * 32) << 16);
       const int m = it.m0 + ml;
       for (int c = 0; c < g.n_pad; c += 32) {
         uint32_t r[32];
         tmem_ld32(taddr + c, r);
         tmem_wait_ld();
+        if (g.cluster) {
+          // this split's partial tile, [n][128 rows] fp32 at the start of the
+          // (drained) stage ring, for the in-cluster reduction below
+          float *tile = reinterpret_cast<float *>(smem);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c + j < g.n_pad) tile[(c + j) * 128 + ml] = __uint_as_float(r[j]);
+          continue;
+        }
         if (m < P.M) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -242,6 +260,43 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
   __syncthreads();
+  if (g.cluster) {
+    // In-cluster split-K reduction: CTA r of the S CTAs of this tile sums rows
+    // [4 q_lo, 4 q_hi) of all S partial tiles (split order 0..S-1, so the sum
+    // is deterministic) and writes the output.
+    cluster_sync();   // every partial tile written
+    const Item it = decode_item(g, item0);
+    const GemmProblem &P = g.p[it.pi];
+    const int S = g.cluster, r = (int)cluster_ctarank();
+    const int q_lo = 32 * r / S, q_hi = 32 * (r + 1) / S, nq = q_hi - q_lo;
+    const uint32_t tile = smem_u32(smem);
+    for (int u = threadIdx.x; u < g.n * nq; u += kThreads) {
+      const int n = u / nq, q = q_lo + u % nq;
+      const int m = it.m0 + 4 * q;
+      if (m >= P.M) continue;
+      const uint32_t off = tile + (uint32_t)((n * 128 + 4 * q) * 4);
+      float4 acc = ld_cluster_v4(mapa(off, 0));
+      for (int sp = 1; sp < S; ++sp) {
+        const float4 v = ld_cluster_v4(mapa(off, (uint32_t)sp));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
+      if (P.out_mode == kOutBf16) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 w;
+        w.x = *reinterpret_cast<uint32_t *>(&lo);
+        w.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(P.out) + idx) = w;
+      } else {
+        *reinterpret_cast<float4 *>(static_cast<float *>(P.out) + idx) = acc;
+      }
+    }
+    cluster_sync();   // no CTA leaves while another still reads its tile
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, g.tmem_cols);
@@ -322,18 +377,38 @@ int gemm_splits(int m_tiles, int heads, int k_chunks) {
   return (k_chunks + per - 1) / per;
 }
 
+int gemm_cluster_splits(int m_tiles, int heads, int k_chunks) {
+  const int s = gemm_splits(m_tiles, heads, k_chunks);
+  if (s <= kMaxClusterSplits) return s;
+  const int per = (k_chunks + kMaxClusterSplits - 1) / kMaxClusterSplits;
+  return (k_chunks + per - 1) / per;
+}
+
 cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, long x_cols, int K,
                  int x_cols_per_head, int *err, cudaStream_t s) {
   if (nops < 1 || nops > 2 || n < 1 || K % 64) return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_sm100_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    if (e != cudaSuccess) return e;
-    attr = true;
+  // in-cluster split-K reduction: every op reduces in clusters of the same size
+  const bool cluster = ops[0].cluster_reduce && !ops[0].part && ops[0].splits > 1;
+  for (int i = 0; i < nops; ++i) {
+    const GemmOp &o = ops[i];
+    if (!cluster) {
+      if (o.cluster_reduce && !o.part && o.splits > 1) return cudaErrorInvalidValue;
+      continue;
+    }
+    if (!o.cluster_reduce || o.part || o.splits != ops[0].splits ||
+        o.splits > kMaxClusterSplits || (o.M % 4) || (o.ldy % 4) || (o.y_head % 4) ||
+        o.out_mode == kOutPartial || (reinterpret_cast<uintptr_t>(o.out) & 15))
+      return cudaErrorInvalidValue;
   }
-  for (int n0 = 0; n0 < n; n0 += 256) {
-    const int nn = n - n0 < 256 ? n - n0 : 256;
+  const int n_step = cluster ? 128 : 256;
+  static api::PerDeviceOnce smem_attr;
+  cudaError_t ea = smem_attr.run([] {
+    return cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                232448);
+  });
+  if (ea != cudaSuccess) return ea;
+  for (int n0 = 0; n0 < n; n0 += n_step) {
+    const int nn = n - n0 < n_step ? n - n0 : n_step;
     GemmLaunch g{};
     g.n = nn;
     g.n0 = n0;
@@ -342,8 +417,9 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     g.k_chunks = K / 64;
     g.x_cols_per_head = x_cols_per_head;
     g.err = err;
+    g.n_cols = (g.n_pad + 31) / 32 * 32;   // accumulator stride: whole 32-column loads
     g.tmem_cols = 32;
-    while (g.tmem_cols < 2 * g.n_pad) g.tmem_cols *= 2;
+    while (g.tmem_cols < 2 * g.n_cols) g.tmem_cols *= 2;
     const int stage_bytes = kABytes + g.n_pad * 128;
     // two CTAs per SM: half of the 227 KB of shared memory each
     g.stages = (232448 / 2 - 1024 - 256) / stage_bytes;
@@ -359,7 +435,7 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
       P.a_mn = o.a_mn;
       P.a_map = i;
       P.a_rows_per_head = o.a_mn ? K : o.M;
-      P.splits = o.part ? o.splits : 1;
+      P.splits = (o.part || cluster) ? o.splits : 1;
       P.chunks_per_split = (g.k_chunks + P.splits - 1) / P.splits;
       P.item_begin = items;
       items += P.m_tiles * P.splits * o.heads;
@@ -380,14 +456,24 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     }
     if (nops == 1) tm[1] = tm[0];
     if (!map2d(&tx, X + (long)n0 * x_cols, nn, x_cols, 64, g.n_pad)) return cudaErrorInvalidValue;
-    // persistent CTAs: at most two per SM, each over a contiguous range of items
-    const int max_ctas = 2 * sm_count();
     g.items = items;
-    g.items_per_cta = (items + max_ctas - 1) / max_ctas;
-    const int ctas = (items + g.items_per_cta - 1) / g.items_per_cta;
     const size_t smem = (size_t)g.stages * stage_bytes + 256 + 1024;
-    cudaError_t e = launch_pdl(gemm_sm100_kernel, dim3(ctas), dim3(kThreads), smem, s, tm[0], tm[1],
-                               tx, g);
+    cudaError_t e;
+    if (cluster) {
+      // one item per CTA; the splits of a tile form one cluster and their
+      // partial tiles ([n_pad][128] fp32) reuse the drained stage ring
+      if ((size_t)g.stages * stage_bytes < (size_t)g.n_pad * 128 * 4) return cudaErrorInvalidValue;
+      g.cluster = ops[0].splits;
+      g.items_per_cta = 1;
+      e = launch_pdl_cluster(gemm_sm100_kernel, dim3(items), dim3(kThreads), smem, s, g.cluster,
+                             tm[0], tm[1], tx, g);
+    } else {
+      // persistent CTAs: at most two per SM, each over a contiguous range of items
+      const int max_ctas = 2 * sm_count();
+      g.items_per_cta = (items + max_ctas - 1) / max_ctas;
+      const int ctas = (items + g.items_per_cta - 1) / g.items_per_cta;
+      e = launch_pdl(gemm_sm100_kernel, dim3(ctas), dim3(kThreads), smem, s, tm[0], tm[1], tx, g);
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -17,6 +17,11 @@ enum : int { kOutPartial = 0, kOutBf16 = 1, kOutF32 = 2 };
 // With part != nullptr the K range is cut into `splits` pieces and each writes
 // fp32 partials part[(split * n_total + n) * part_ld + part_col + head * M + m];
 // gemm_reduce sums them.
+// With cluster_reduce (part == nullptr, 2 <= splits <= kMaxClusterSplits, M,
+// ldy and y_head multiples of 4) the `splits` CTAs of one tile form a thread-
+// block cluster and sum their partial tiles through distributed shared memory
+// in a fixed order, writing the direct output; no partial buffer, no reduce
+// launch.  Every op of a launch must then use the same splits.
 struct GemmOp {
   const __nv_bfloat16 *A;
   int M, heads, a_mn;
@@ -25,7 +30,10 @@ struct GemmOp {
   long ldy, y_head;
   float *part;
   int part_ld, part_col, splits;
+  int cluster_reduce;
 };
+
+constexpr int kMaxClusterSplits = 8;
 
 // Kernel-side description of one problem of a launch.  Its work items are
 // (head, split, m_tile) triples numbered from item_begin.
@@ -39,10 +47,14 @@ struct GemmProblem {
 
 struct GemmLaunch {
   GemmProblem p[2];
-  int nprob, n, n0, n_total, n_pad, k_chunks, x_cols_per_head, stages, tmem_cols;
+  int nprob, n, n0, n_total, n_pad, n_cols, k_chunks, x_cols_per_head, stages, tmem_cols;
   int items, items_per_cta;
+  int cluster;  // CTAs per cluster (the splits of one tile) in cluster-reduce mode, else 0
   int *err;
 };
+
+// Split count for an in-cluster reduction (at most kMaxClusterSplits).
+int gemm_cluster_splits(int m_tiles, int heads, int k_chunks);
 
 // Split count for a problem of m_tiles x heads tiles and K / 64 chunks.
 int gemm_splits(int m_tiles, int heads, int k_chunks);

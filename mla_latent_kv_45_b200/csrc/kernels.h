@@ -40,6 +40,7 @@ struct PlanArgs {
   const int32_t *seq_lens;
   int batch, page_size, max_pages;
   int parts_max, min_pages;
+  int allow_empty;  // seq_len == 0 is an empty share (no rows), not an error
   PlanHeader *hdr;
   int *seq_start;  // [batch + 1]
   int *part_base;  // [batch]
@@ -66,6 +67,9 @@ struct AttnArgs {
   float *part_m;  // [slots][n_heads]
   float *part_l;  // [slots][n_heads]
   int *err;
+  // Partial-softmax output (nullptr for z / lse): unnormalised O [batch][n_heads][d_c],
+  // m (natural-log max) and l [batch][n_heads], fp32.
+  float *pout_O, *pout_m, *pout_l;
 };
 
 template <class T>
@@ -73,6 +77,15 @@ cudaError_t launch_attn_simt(const AttnArgs &a, int parts_max, cudaStream_t s);
 
 template <class T>
 cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s);
+
+// Merge of n partial softmaxes (unnormalised O, natural-log m, l), laid out
+// [n][batch][n_heads](*d_c): z = sum_j w_j O_j / sum_j w_j l_j, w_j = e^(m_j - max m),
+// lse = max m + log(sum_j w_j l_j); rows whose parts are all empty get z = 0,
+// lse = -inf.
+template <class T>
+cudaError_t launch_merge_partials(const float *O, const float *m, const float *l, int n_parts,
+                                  int batch, int n_heads, int d_c, T *z, float *lse,
+                                  cudaStream_t s);
 
 }  // namespace mla
 

@@ -249,7 +249,8 @@ __global__ void plan_kernel(PlanArgs a) {
       const bool ok = len > 0 && len <= cap;
       n = ok ? (len + a.page_size - 1) / a.page_size : 0;
       a.bad[b] = ok ? 0 : 1;
-      if (!ok) set_error(a.err, kErrRange);
+      // an empty share of a sequence split across devices is not an error
+      if (!ok && !(a.allow_empty && len == 0)) set_error(a.err, kErrRange);
     }
     // block-wide inclusive scan of n
     int v = n;
@@ -422,7 +423,18 @@ __global__ void attn_simt(AttnArgs a) {
       __syncthreads();
     }
     const int pb = a.part_base[b];
-    if (pb < 0) {
+    if (pb < 0 && a.pout_O) {
+      float *O = a.pout_O + ((long)b * a.n_heads + h) * a.d_c;
+#pragma unroll
+      for (int k = 0; k < MAXD; ++k) {
+        const int d = threadIdx.x + k * NT;
+        if (d < a.d_c) O[d] = acc[k];
+      }
+      if (threadIdx.x == 0) {
+        a.pout_m[(long)b * a.n_heads + h] = m;
+        a.pout_l[(long)b * a.n_heads + h] = l;
+      }
+    } else if (pb < 0) {
       T *z = reinterpret_cast<T *>(a.z) + ((long)b * a.n_heads + h) * a.d_c;
       const float inv = 1.f / l;
 #pragma unroll
@@ -497,7 +509,18 @@ __global__ void combine_kernel(AttnArgs a) {
   if (row >= a.batch * a.n_heads) return;
   const int b = row / a.n_heads, h = row % a.n_heads;
   T *zr = reinterpret_cast<T *>(a.z) + (long)row * a.d_c;
+  float *por = a.pout_O ? a.pout_O + (long)row * a.d_c : nullptr;
   if (a.bad[b]) {
+    // no rows (an error, or an empty share): z = 0, lse = -inf; as a partial,
+    // O = 0, m = -inf, l = 0 (it then carries no weight in a merge)
+    if (por) {
+      for (int d = lane; d < a.d_c; d += 32) por[d] = 0.f;
+      if (lane == 0) {
+        a.pout_m[row] = -INFINITY;
+        a.pout_l[row] = 0.f;
+      }
+      return;
+    }
     for (int d = lane; d < a.d_c; d += 32) zr[d] = st_cast<T>(0.f);
     if (a.lse && lane == 0) a.lse[row] = -INFINITY;
     return;
@@ -519,8 +542,13 @@ __global__ void combine_kernel(AttnArgs a) {
     den += expf(__ldcg(pm + (long)j * a.n_heads) - M) * __ldcg(pl + (long)j * a.n_heads);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-  const float inv = 1.f / den;
-  if (a.lse && lane == 0) a.lse[row] = M + logf(den);
+  // as a partial: O = sum_j e^(m_j - M) O_j, m = M, l = den (not normalised)
+  const float inv = por ? 1.f : 1.f / den;
+  if (por && lane == 0) {
+    a.pout_m[row] = M;
+    a.pout_l[row] = den;
+  }
+  if (!por && a.lse && lane == 0) a.lse[row] = M + logf(den);
   const int nvec = a.d_c / 4;
   const float4 *src = reinterpret_cast<const float4 *>(a.part_O + ((long)pb * a.n_heads + h) * a.d_c);
   const long piece_stride = (long)a.n_heads * nvec;   // float4 per piece
@@ -555,7 +583,11 @@ __global__ void combine_kernel(AttnArgs a) {
 #pragma unroll
     for (int q = 0; q < kCombineVecs; ++q) {
       const int vi = v0 + lane + 32 * q;
-      if (vi < nvec) Vec4Out<T>::store(zr + 4 * vi, acc[q]);
+      if (vi >= nvec) continue;
+      if (por)
+        *reinterpret_cast<float4 *>(por + 4 * vi) = acc[q];
+      else
+        Vec4Out<T>::store(zr + 4 * vi, acc[q]);
     }
   }
 }
@@ -570,5 +602,57 @@ cudaError_t launch_combine(const AttnArgs &a, cudaStream_t s) {
 }
 template cudaError_t launch_combine<float>(const AttnArgs &, cudaStream_t);
 template cudaError_t launch_combine<__nv_bfloat16>(const AttnArgs &, cudaStream_t);
+
+// Merge of n partial softmaxes [n][batch][n_heads](*d_c): one warp per
+// (sequence, head) row, parts summed in increasing order.
+template <class T>
+__global__ void merge_partials_kernel(const float *O, const float *m, const float *l, int n_parts,
+                                      int rows, int d_c, T *z, float *lse) {
+  grid_dep_wait();
+  grid_dep_launch();
+  const int row = blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float M = -INFINITY;
+  for (int j = lane; j < n_parts; j += 32) M = fmaxf(M, m[(long)j * rows + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  T *zr = z + (long)row * d_c;
+  if (M == -INFINITY) {   // every part empty
+    for (int d = lane; d < d_c; d += 32) zr[d] = st_cast<T>(0.f);
+    if (lse && lane == 0) lse[row] = -INFINITY;
+    return;
+  }
+  float den = 0.f;
+  for (int j = lane; j < n_parts; j += 32)
+    den += expf(m[(long)j * rows + row] - M) * l[(long)j * rows + row];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lse && lane == 0) lse[row] = M + logf(den);
+  const float inv = 1.f / den;
+  for (int d = lane; d < d_c; d += 32) {
+    float acc = 0.f;
+    for (int j = 0; j < n_parts; ++j)
+      acc = fmaf(expf(m[(long)j * rows + row] - M) * inv, O[((long)j * rows + row) * d_c + d], acc);
+    zr[d] = st_cast<T>(acc);
+  }
+}
+
+template <class T>
+cudaError_t launch_merge_partials(const float *O, const float *m, const float *l, int n_parts,
+                                  int batch, int n_heads, int d_c, T *z, float *lse,
+                                  cudaStream_t s) {
+  const int rows = batch * n_heads;
+  const dim3 grid((rows + kCombineWarps - 1) / kCombineWarps);
+  cudaError_t e = launch_pdl(merge_partials_kernel<T>, grid, dim3(32 * kCombineWarps), 0, s, O, m,
+                             l, n_parts, rows, d_c, z, lse);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+template cudaError_t launch_merge_partials<float>(const float *, const float *, const float *, int,
+                                                  int, int, int, float *, float *, cudaStream_t);
+template cudaError_t launch_merge_partials<__nv_bfloat16>(const float *, const float *,
+                                                          const float *, int, int, int, int,
+                                                          __nv_bfloat16 *, float *, cudaStream_t);
 
 }  // namespace mla

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "mla.h"
+#include "api_checks.h"
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.h"
@@ -14,6 +15,10 @@
 namespace {
 
 using namespace mla;
+using api::aligned16;
+using api::check_cache;
+using api::check_dims;
+using api::softmax_scale;
 using bf16 = __nv_bfloat16;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -21,8 +26,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Workspace regions (byte offsets).  The first 256 bytes hold the device
 // error word (offset 0) and the attention plan header (offset 64).
 struct Layout {
-  size_t err, hdr, seq_start, part_base, bad, part_O, part_m, part_l, xkv, cq, qc, qr, o, gemm,
-      total;
+  size_t err, hdr, seq_start, part_base, bad, part_O, part_m, part_l, xkv, cq, qc, qr, o, total;
   int slots;
 };
 
@@ -63,46 +67,14 @@ Layout make_layout(const mla_dims &d, int batch, int d_model, int d_q, int parts
   L.qc = off; off = align256(off + sizeof(float) * (size_t)batch * H * d.d_nope);
   L.qr = off; off = align256(off + sizeof(float) * (size_t)batch * H * d.d_rope);
   L.o = off; off = align256(off + sizeof(float) * (size_t)batch * H * d.d_v);
-  L.gemm = off; off = align256(off + sm100::gemm_workspace_bytes(batch, d_model, d_q, H, d));
   L.total = off;
   (void)d_model;
   return L;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-mla_status check_dims(const mla_dims *d) {
-  if (!d) return MLA_ERR_INVALID_ARG;
-  if (d->n_heads < 1 || d->d_c < 1 || d->d_nope < 1 || d->d_v < 1 || d->page_size < 1)
-    return MLA_ERR_INVALID_ARG;
-  if (d->d_rope < 2 || (d->d_rope & 1) || d->d_rope > 128) return MLA_ERR_INVALID_ARG;
-  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32) return MLA_ERR_INVALID_ARG;
-  if (d->rope_layout != MLA_ROPE_INTERLEAVED && d->rope_layout != MLA_ROPE_HALF)
-    return MLA_ERR_INVALID_ARG;
-  if (!(d->rope_base > 0.0) || !(d->rms_eps >= 0.0) || !(d->softmax_scale >= 0.0))
-    return MLA_ERR_INVALID_ARG;
-  if (d->dtype == MLA_FP32) {
-    if (d->n_heads > 256 || d->d_c > 1024 || (d->d_c % 4) || d->d_nope > 256 || d->d_v > 256)
-      return MLA_ERR_UNSUPPORTED;
-  } else {
-    if (d->n_heads != 128 || d->d_c != 512 || d->d_rope != 64 || d->d_nope != 128 ||
-        d->d_v != 128 || d->page_size != 64)
-      return MLA_ERR_UNSUPPORTED;
-  }
-  return MLA_OK;
-}
-
 mla_status check_width(const mla_dims *d, int w) {
   if (w < 1) return MLA_ERR_INVALID_ARG;
   if (d->dtype == MLA_BF16 && (w % 64)) return MLA_ERR_UNSUPPORTED;
-  return MLA_OK;
-}
-
-mla_status check_cache(const mla_paged_cache *c) {
-  if (!c || !c->pool || !c->block_table || c->num_pages < 1 || c->max_pages_per_seq < 1)
-    return MLA_ERR_INVALID_ARG;
-  if (!aligned16(c->pool) || (reinterpret_cast<uintptr_t>(c->block_table) & 3))
-    return MLA_ERR_ALIGNMENT;
   return MLA_OK;
 }
 
@@ -113,10 +85,6 @@ RopeParams rope_params(const mla_dims &d) {
   rp.half = d.rope_layout == MLA_ROPE_HALF;
   for (int i = 0; i < d.d_rope / 2; ++i) rp.theta[i] = pow(d.rope_base, -2.0 * i / d.d_rope);
   return rp;
-}
-
-float softmax_scale(const mla_dims &d) {
-  return d.softmax_scale > 0 ? (float)d.softmax_scale : (float)(1.0 / sqrt((double)(d.d_nope + d.d_rope)));
 }
 
 char *at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
@@ -135,6 +103,66 @@ mla_status gemv(const void *W, long w_head, long w_m, long w_k, const void *X, l
                 cudaStream_t s) {
   GemvArgs a{W, w_head, w_m, w_k, X, x_head, x_b, Y, y_head, y_b, M, K, B};
   return cuda_ok(launch_gemv<TW, TX, TY>(a, heads, s));
+}
+
+// Plan, attention and merge: z / lse, or with pO the unnormalised partial
+// softmax (O, m, l) of the rows the cache holds.  Arguments already checked.
+mla_status decode_attn_impl(const mla_dims *dims, const mla_paged_cache *cache, int batch,
+                            const void *q_lat, void *z, float *lse, float *pO, float *pm,
+                            float *pl, int num_splits, void *ws, size_t ws_bytes,
+                            cudaStream_t s) {
+  if (!ws) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MLA_ERR_ALIGNMENT;
+  const mla_dims &d = *dims;
+  const int parts = parts_for(d, num_splits);
+  const Layout L = make_layout(d, batch, 64, 0, parts);
+  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
+  PlanArgs pa{};
+  pa.seq_lens = cache->seq_lens;
+  pa.batch = batch;
+  pa.page_size = d.page_size;
+  pa.max_pages = cache->max_pages_per_seq;
+  pa.parts_max = parts;
+  pa.min_pages = d.dtype == MLA_BF16 ? sm100::kAttnMinPages : 1;
+  pa.allow_empty = pO != nullptr;
+  pa.hdr = reinterpret_cast<PlanHeader *>(at(ws, L.hdr));
+  pa.seq_start = reinterpret_cast<int *>(at(ws, L.seq_start));
+  pa.part_base = reinterpret_cast<int *>(at(ws, L.part_base));
+  pa.bad = reinterpret_cast<int *>(at(ws, L.bad));
+  pa.err = reinterpret_cast<int *>(at(ws, L.err));
+  MLA_TRY(cuda_ok(launch_plan(pa, s)));
+  AttnArgs a{};
+  a.q_lat = q_lat;
+  a.pool = cache->pool;
+  a.block_table = cache->block_table;
+  a.seq_lens = cache->seq_lens;
+  a.z = z;
+  a.lse = lse;
+  a.batch = batch;
+  a.n_heads = d.n_heads;
+  a.d_c = d.d_c;
+  a.d_rope = d.d_rope;
+  a.page_size = d.page_size;
+  a.num_pages = cache->num_pages;
+  a.max_pages = cache->max_pages_per_seq;
+  a.scale = softmax_scale(d);
+  a.hdr = pa.hdr;
+  a.seq_start = pa.seq_start;
+  a.part_base = pa.part_base;
+  a.bad = pa.bad;
+  a.part_O = reinterpret_cast<float *>(at(ws, L.part_O));
+  a.part_m = reinterpret_cast<float *>(at(ws, L.part_m));
+  a.part_l = reinterpret_cast<float *>(at(ws, L.part_l));
+  a.err = pa.err;
+  a.pout_O = pO;
+  a.pout_m = pm;
+  a.pout_l = pl;
+  if (d.dtype == MLA_FP32) {
+    MLA_TRY(cuda_ok(launch_attn_simt<float>(a, parts, s)));
+    return cuda_ok(launch_combine<float>(a, s));
+  }
+  MLA_TRY(cuda_ok(sm100::launch_attn(a, parts, s)));
+  return cuda_ok(launch_combine<bf16>(a, s));
 }
 
 }  // namespace
@@ -184,13 +212,11 @@ mla_status mla_cache_append(const mla_dims *dims, const mla_paged_cache *cache, 
         static_cast<float *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
         cache->max_pages_per_seq, err, s));
   }
-  const float *parts = nullptr;
-  int splits = 1;
   MLA_TRY(cuda_ok(sm100::append_proj(static_cast<const bf16 *>(h), static_cast<const bf16 *>(W_DKV),
-                                     static_cast<const bf16 *>(W_KR), batch, d_model, xkv,
-                                     at(ws, L.gemm), err, &parts, &splits, s)));
+                                     static_cast<const bf16 *>(W_KR), batch, d_model, xkv, err,
+                                     s)));
   return cuda_ok(launch_append_finish<bf16>(
-      parts, splits, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
+      xkv, 1, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
       static_cast<bf16 *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
       cache->max_pages_per_seq, err, s));
 }
@@ -240,74 +266,48 @@ mla_status mla_absorb_q(const mla_dims *dims, int batch, int d_in, const void *x
     return cuda_ok(launch_rope_q<float>(qr, batch, H, d.d_c, rp, positions,
                                         static_cast<float *>(q_lat), s));
   }
-  MLA_TRY(cuda_ok(sm100::absorb_proj(
+  return cuda_ok(sm100::absorb_proj(
       static_cast<const bf16 *>(x), static_cast<const bf16 *>(W_DQ),
       static_cast<const bf16 *>(W_UQ), static_cast<const bf16 *>(W_QR),
-      static_cast<const bf16 *>(W_UK), batch, d_in, d_q, reinterpret_cast<bf16 *>(cq),
-      reinterpret_cast<bf16 *>(qc), qr, static_cast<bf16 *>(q_lat), at(ws, L.gemm),
-      reinterpret_cast<int *>(at(ws, L.err)), s)));
-  return cuda_ok(launch_rope_q<bf16>(qr, batch, H, d.d_c, rp, positions,
-                                     static_cast<bf16 *>(q_lat), s));
+      static_cast<const bf16 *>(W_UK), batch, d_in, d_q, rp, positions,
+      reinterpret_cast<bf16 *>(cq), static_cast<bf16 *>(q_lat),
+      reinterpret_cast<int *>(at(ws, L.err)), s));
 }
 
 mla_status mla_decode_attn(const mla_dims *dims, const mla_paged_cache *cache, int batch,
                            const void *q_lat, void *z, float *lse, int num_splits, void *ws,
                            size_t ws_bytes, mla_stream_t stream) {
+  MLA_TRY(api::check_attn_args(dims, cache, batch, q_lat, z, lse, num_splits));
+  return decode_attn_impl(dims, cache, batch, q_lat, z, lse, nullptr, nullptr, nullptr,
+                          num_splits, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+mla_status mla_decode_attn_partial(const mla_dims *dims, const mla_paged_cache *cache, int batch,
+                                   const void *q_lat, float *O, float *m, float *l, int num_splits,
+                                   void *ws, size_t ws_bytes, mla_stream_t stream) {
+  if (!O || !m || !l) return MLA_ERR_INVALID_ARG;
+  // O takes z's place in the argument rules (16-byte aligned); m and l are fp32 like lse
+  MLA_TRY(api::check_attn_args(dims, cache, batch, q_lat, O, m, num_splits));
+  if (!api::aligned4(l)) return MLA_ERR_ALIGNMENT;
+  return decode_attn_impl(dims, cache, batch, q_lat, nullptr, nullptr, O, m, l, num_splits, ws,
+                          ws_bytes, (cudaStream_t)stream);
+}
+
+mla_status mla_merge_partials(const mla_dims *dims, int batch, int n_parts, const float *O,
+                              const float *m, const float *l, void *z, float *lse,
+                              mla_stream_t stream) {
   MLA_TRY(check_dims(dims));
-  MLA_TRY(check_cache(cache));
-  if (batch < 1 || !q_lat || !z || !ws || !cache->seq_lens || num_splits < 0)
-    return MLA_ERR_INVALID_ARG;
-  if (!aligned16(q_lat) || !aligned16(z) || !aligned16(ws) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) ||
-      (reinterpret_cast<uintptr_t>(cache->seq_lens) & 3))
+  if (batch < 1 || n_parts < 1 || !O || !m || !l || !z) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(O) || !api::aligned4(m) || !api::aligned4(l) || !aligned16(z) ||
+      (lse && !api::aligned4(lse)))
     return MLA_ERR_ALIGNMENT;
   const mla_dims &d = *dims;
-  const int parts = parts_for(d, num_splits);
-  const Layout L = make_layout(d, batch, 64, 0, parts);
-  if (ws_bytes < L.total) return MLA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
-  PlanArgs pa;
-  pa.seq_lens = cache->seq_lens;
-  pa.batch = batch;
-  pa.page_size = d.page_size;
-  pa.max_pages = cache->max_pages_per_seq;
-  pa.parts_max = parts;
-  pa.min_pages = d.dtype == MLA_BF16 ? sm100::kAttnMinPages : 1;
-  pa.hdr = reinterpret_cast<PlanHeader *>(at(ws, L.hdr));
-  pa.seq_start = reinterpret_cast<int *>(at(ws, L.seq_start));
-  pa.part_base = reinterpret_cast<int *>(at(ws, L.part_base));
-  pa.bad = reinterpret_cast<int *>(at(ws, L.bad));
-  pa.err = reinterpret_cast<int *>(at(ws, L.err));
-  MLA_TRY(cuda_ok(launch_plan(pa, s)));
-  AttnArgs a;
-  a.q_lat = q_lat;
-  a.pool = cache->pool;
-  a.block_table = cache->block_table;
-  a.seq_lens = cache->seq_lens;
-  a.z = z;
-  a.lse = lse;
-  a.batch = batch;
-  a.n_heads = d.n_heads;
-  a.d_c = d.d_c;
-  a.d_rope = d.d_rope;
-  a.page_size = d.page_size;
-  a.num_pages = cache->num_pages;
-  a.max_pages = cache->max_pages_per_seq;
-  a.scale = softmax_scale(d);
-  a.hdr = pa.hdr;
-  a.seq_start = pa.seq_start;
-  a.part_base = pa.part_base;
-  a.bad = pa.bad;
-  a.part_O = reinterpret_cast<float *>(at(ws, L.part_O));
-  a.part_m = reinterpret_cast<float *>(at(ws, L.part_m));
-  a.part_l = reinterpret_cast<float *>(at(ws, L.part_l));
-  a.err = pa.err;
-  if (d.dtype == MLA_FP32) {
-    MLA_TRY(cuda_ok(launch_attn_simt<float>(a, parts, s)));
-    return cuda_ok(launch_combine<float>(a, s));
-  }
-  MLA_TRY(cuda_ok(sm100::launch_attn(a, parts, s)));
-  return cuda_ok(launch_combine<bf16>(a, s));
+  if (d.dtype == MLA_FP32)
+    return cuda_ok(launch_merge_partials<float>(O, m, l, n_parts, batch, d.n_heads, d.d_c,
+                                               static_cast<float *>(z), lse, s));
+  return cuda_ok(launch_merge_partials<bf16>(O, m, l, n_parts, batch, d.n_heads, d.d_c,
+                                            static_cast<bf16 *>(z), lse, s));
 }
 
 mla_status mla_unabsorb_out(const mla_dims *dims, int batch, const void *z, const void *W_UV,
@@ -336,7 +336,7 @@ mla_status mla_unabsorb_out(const mla_dims *dims, int batch, const void *z, cons
   }
   return cuda_ok(sm100::unabsorb_proj(
       static_cast<const bf16 *>(z), static_cast<const bf16 *>(W_UV), static_cast<const bf16 *>(W_O),
-      batch, d_model, reinterpret_cast<bf16 *>(o), static_cast<bf16 *>(out), at(ws, L.gemm),
+      batch, d_model, reinterpret_cast<bf16 *>(o), static_cast<bf16 *>(out),
       reinterpret_cast<int *>(at(ws, L.err)), s));
 }
 
@@ -351,6 +351,12 @@ mla_status mla_get_device_error(void *ws, mla_stream_t stream) {
     return MLA_ERR_CUDA;
   if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
   if (word & kErrRange) return MLA_ERR_DEVICE_RANGE;
+  return MLA_OK;
+}
+
+mla_status mla_debug_absorb_timeout(int enable, unsigned wait_limit_us) {
+  if (enable && wait_limit_us == 0) return MLA_ERR_INVALID_ARG;
+  sm100::absorb_debug_fault(enable ? 1 : 0, enable ? (uint64_t)wait_limit_us * 1000ull : 0);
   return MLA_OK;
 }
 

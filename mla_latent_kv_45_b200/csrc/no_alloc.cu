@@ -17,11 +17,17 @@
 // stream capture.  All calls share the one array: two calls whose work
 // overlaps on the GPU (different streams, or different host threads on the
 // same device) race on it and must be serialised by the caller.
+//
+// The error word of the scratch is cleared at the start of each call and
+// records what the device saw during it (a page entry, length or position out
+// of range, or a bounded wait that gave up); mla_noalloc_get_device_error waits
+// for the stream and reads and clears it.
 #include <cuda_runtime.h>
 #include <math.h>
 
 #include <mutex>
 
+#include "api_checks.h"
 #include "common.cuh"
 #include "kernels.h"
 #include "mla.h"
@@ -77,35 +83,15 @@ mla_status scratch_address(void **out) {
   return MLA_OK;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
 }  // namespace
 
 extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_paged_cache *cache,
                                               int batch, const void *q_lat, void *z, float *lse,
                                               int num_splits, mla_stream_t stream) {
-  if (!dims || !cache || !cache->pool || !cache->block_table || !cache->seq_lens || !q_lat ||
-      !z || batch < 1 || num_splits < 0 || cache->num_pages < 1 || cache->max_pages_per_seq < 1)
-    return MLA_ERR_INVALID_ARG;
+  // the same argument rules as mla_decode_attn
+  const mla_status chk = api::check_attn_args(dims, cache, batch, q_lat, z, lse, num_splits);
+  if (chk != MLA_OK) return chk;
   const mla_dims &d = *dims;
-  // the same shape rules as mla_decode_attn
-  if (d.n_heads < 1 || d.d_c < 1 || d.d_nope < 1 || d.d_v < 1 || d.page_size < 1 ||
-      d.d_rope < 2 || (d.d_rope & 1) || d.d_rope > 128 || !(d.rope_base > 0.0) ||
-      !(d.rms_eps >= 0.0) || !(d.softmax_scale >= 0.0) ||
-      (d.dtype != MLA_BF16 && d.dtype != MLA_FP32) ||
-      (d.rope_layout != MLA_ROPE_INTERLEAVED && d.rope_layout != MLA_ROPE_HALF))
-    return MLA_ERR_INVALID_ARG;
-  if (d.dtype == MLA_FP32 &&
-      (d.n_heads > 256 || d.d_c > 1024 || (d.d_c % 4) || d.d_nope > 256 || d.d_v > 256))
-    return MLA_ERR_UNSUPPORTED;
-  if (d.dtype == MLA_BF16 && (d.n_heads != 128 || d.d_c != 512 || d.d_rope != 64 ||
-                              d.d_nope != 128 || d.d_v != 128 || d.page_size != 64))
-    return MLA_ERR_UNSUPPORTED;
-  if (!aligned16(q_lat) || !aligned16(z) || !aligned16(cache->pool) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) ||
-      (reinterpret_cast<uintptr_t>(cache->seq_lens) & 3) ||
-      (reinterpret_cast<uintptr_t>(cache->block_table) & 3))
-    return MLA_ERR_ALIGNMENT;
 
   // partitions: as requested, or (0) the most that fit, at most one per SM pair
   int parts = num_splits;
@@ -128,7 +114,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
   // before it is read
   if (cudaMemsetAsync(ws, 0, 256, s) != cudaSuccess) return MLA_ERR_CUDA;
 
-  PlanArgs pa;
+  PlanArgs pa{};
   pa.seq_lens = cache->seq_lens;
   pa.batch = batch;
   pa.page_size = d.page_size;
@@ -142,7 +128,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
   pa.err = reinterpret_cast<int *>(ws + R.err);
   if (launch_plan(pa, s) != cudaSuccess) return MLA_ERR_CUDA;
 
-  AttnArgs a;
+  AttnArgs a{};
   a.q_lat = q_lat;
   a.pool = cache->pool;
   a.block_table = cache->block_table;
@@ -156,8 +142,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
   a.page_size = d.page_size;
   a.num_pages = cache->num_pages;
   a.max_pages = cache->max_pages_per_seq;
-  a.scale = d.softmax_scale > 0 ? (float)d.softmax_scale
-                                : (float)(1.0 / sqrt((double)(d.d_nope + d.d_rope)));
+  a.scale = api::softmax_scale(d);
   a.hdr = pa.hdr;
   a.seq_start = pa.seq_start;
   a.part_base = pa.part_base;
@@ -175,4 +160,20 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
     if (e == cudaSuccess) e = launch_combine<__nv_bfloat16>(a, s);
   }
   return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+extern "C" mla_status mla_noalloc_get_device_error(mla_stream_t stream) {
+  void *base = nullptr;
+  const mla_status st = scratch_address(&base);
+  if (st != MLA_OK) return st;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MLA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, base, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(base, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (word & kErrTimeout) return MLA_ERR_TIMEOUT;
+  if (word & kErrRange) return MLA_ERR_DEVICE_RANGE;
+  return MLA_OK;
 }

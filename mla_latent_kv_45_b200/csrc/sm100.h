@@ -16,28 +16,36 @@ namespace sm100 {
 // less work than this is merged away by the plan).
 constexpr int kAttnMinPages = 4;
 
-// Workspace bytes the projections need beyond the fp32 intermediates.
-size_t gemm_workspace_bytes(int batch, int d_model, int d_q, int n_heads, const mla_dims &d);
-
-// [W_DKV h_b ; W_KR h_b] in fp32 as `*splits` partial sums [splits][batch][576]
-// at *out (xkv itself when there is one split, else the GEMM workspace).
+// [W_DKV h_b ; W_KR h_b] in fp32 into xkv [batch][576].
 cudaError_t append_proj(const __nv_bfloat16 *h, const __nv_bfloat16 *W_DKV,
-                        const __nv_bfloat16 *W_KR, int batch, int d_model, float *xkv,
-                        void *gemm_ws, int *err, const float **out, int *splits,
+                        const __nv_bfloat16 *W_KR, int batch, int d_model, float *xkv, int *err,
                         cudaStream_t s);
 
-// c_Q (bf16, when W_DQ), q_C (bf16), raw q_R (fp32, not yet rotated) and the
-// absorbed content half q_lat[b][i][0:512] = W_UK,i^T q_C,i (bf16).
+// q_lat[b][i] = [W_UK,i^T q_C,i ; RoPE_pos(q_R,i)] (bf16), with c_Q = W_DQ x
+// (bf16, in cq) when W_DQ is given, else c_Q = x.
 cudaError_t absorb_proj(const __nv_bfloat16 *x, const __nv_bfloat16 *W_DQ,
                         const __nv_bfloat16 *W_UQ, const __nv_bfloat16 *W_QR,
                         const __nv_bfloat16 *W_UK, int batch, int d_in, int d_q,
-                        __nv_bfloat16 *cq, __nv_bfloat16 *qc, float *qr, __nv_bfloat16 *q_lat,
-                        void *gemm_ws, int *err, cudaStream_t s);
+                        const RopeParams &rp, const int32_t *positions, __nv_bfloat16 *cq,
+                        __nv_bfloat16 *q_lat, int *err, cudaStream_t s);
+
+// The per-head part of absorb_proj in one launch (one CTA per head): q_C,i =
+// W_UQ,i x (rounded to bf16), q_R,i = W_QR,i x rotated by positions[b], and
+// q~_i = W_UK,i^T q_C,i, written into q_lat.  x: [batch][K] bf16.
+cudaError_t absorb_heads(const __nv_bfloat16 *x, int K, const __nv_bfloat16 *W_UQ,
+                         const __nv_bfloat16 *W_QR, const __nv_bfloat16 *W_UK, int batch,
+                         const RopeParams &rp, const int32_t *positions, __nv_bfloat16 *q_lat,
+                         int *err, cudaStream_t s);
 
 // o[b][i] = W_UV,i z[b][i] (bf16); out = W_O o when W_O is given, else out = o.
 cudaError_t unabsorb_proj(const __nv_bfloat16 *z, const __nv_bfloat16 *W_UV,
                           const __nv_bfloat16 *W_O, int batch, int d_model, __nv_bfloat16 *o,
-                          __nv_bfloat16 *out, void *gemm_ws, int *err, cudaStream_t s);
+                          __nv_bfloat16 *out, int *err, cudaStream_t s);
+
+// Test hook: when limit_ns > 0, later absorb_heads launches bound every wait
+// by limit_ns instead of the default, and with skip_arrive one epilogue warp
+// withholds its arrive on the q_C-ready barrier (so that wait runs out).
+void absorb_debug_fault(int skip_arrive, uint64_t limit_ns);
 
 // Latent attention over the plan's partitions (partials / z / lse).
 cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s);

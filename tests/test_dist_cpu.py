@@ -76,3 +76,23 @@ def test_stored_traffic_only_for_the_captured_sources(tmp_path):
                              "dram_bytes_per_launch": 123}))
     assert bench.stored_traffic("v2_batch64", str(f)) is None
     assert bench.stored_traffic("v2_batch64", str(tmp_path / "missing.json")) is None
+
+
+def test_bench_gpus_flag_starts_ranks():
+    """``bench.py --gpus 2`` outside torchrun starts two ranks itself; the
+    plumbing check runs them on CPU (gloo) through the same max-over-ranks
+    reduction, and rank 0 alone prints one line with n_gpus = 2."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--rank-check"], capture_output=True, text=True, timeout=300,
+                       env={**os.environ, "OMP_NUM_THREADS": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    # the max over ranks of 1 + rank, and of the ranks' workload seeds (base + 100 rank)
+    import bench
+    assert lines[0] == {"n_gpus": 2, "max_ms": 2.0,
+                        "max_wid": float(bench.workload("v2_batch64", 1).wid)}

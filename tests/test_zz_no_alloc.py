@@ -5,9 +5,11 @@ memory is fully owned by another allocator, and plugin interfaces that pass
 only the operation's tensors and allow no allocation while it runs.  Its
 scratch is a fixed array inside the library, so nothing here hands it a
 workspace.  Each case calls it twice in a row through the C ABI and checks
-both results against mla_decode_attn (which takes a caller workspace) on the
-same inputs, within the tolerances the parity tests use.  This file is named to
-be collected last; it needs no state from other tests.
+both results element by element against the fp64 oracle, and against
+mla_decode_attn (which takes a caller workspace) on the same inputs, within the
+tolerances the parity tests use.  Its device status is read back with
+mla_noalloc_get_device_error.  This file is named to be collected last; it
+needs no state from other tests.
 """
 
 import ctypes
@@ -17,10 +19,12 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mla_latent_kv_45_b200 import _lib as L
 from mla_latent_kv_45_b200 import build, synth
 
-from mla_testlib import assert_bf16_close, assert_fp32_close, dev, dev_cache, host, lib_dims
+from mla_testlib import (assert_bf16_close, assert_fp32_close, dev, dev_cache, host, lib_dims,
+                         oracle_dims)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,8 +55,12 @@ def _noalloc_c_abi(dims, cache, q, z, lse, splits=0):
                                            torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("kind", ["bf16", "fp32"])
-def test_noalloc_matches_workspace_entry_point(kind):
+def _noalloc_status():
+    return L.lib().mla_noalloc_get_device_error(torch.cuda.current_stream().cuda_stream)
+
+
+@pytest.mark.parametrize("kind,splits", [("bf16", 0), ("bf16", 7), ("fp32", 0)])
+def test_noalloc_matches_oracle_and_workspace_entry_point(kind, splits):
     if kind == "bf16":
         lens = np.array([1, 700, 5000, 64, 3000, 129])
         wl = synth.reduced(synth.V2_BATCH64, "noalloc_bf16", 50, len(lens), 0, 0, new_tokens=0)
@@ -63,19 +71,46 @@ def test_noalloc_matches_workspace_entry_point(kind):
                                  new_tokens=0)
         close = assert_fp32_close
     pc = synth.make_paged_cache(wl, lens, spare_pages=1)
-    q = dev(synth.make_q_lat(wl), wl)
+    q_host = synth.make_q_lat(wl)
+    q = dev(q_host, wl)
     dims = lib_dims(wl)
     cache = dev_cache(pc, lens)
-    z_ref, lse_ref = _with_workspace(dims, cache, q, wl.batch)
-    z = torch.empty_like(z_ref)
-    lse = torch.empty_like(lse_ref)
+    od = oracle_dims(wl)
+    ref = [oracle.attend_latent(q_host[b], pc.rows_f32(b, Lb), od) for b, Lb in enumerate(lens)]
+    z_ws, lse_ws = _with_workspace(dims, cache, q, wl.batch, splits)
+    z = torch.empty_like(z_ws)
+    lse = torch.empty_like(lse_ws)
     for call in range(2):
         z.fill_(3.0)
         lse.fill_(3.0)
-        assert _noalloc_c_abi(dims, cache, q, z, lse) == 0
-        torch.cuda.synchronize()
-        close(host(z), host(z_ref), f"z, call {call}")
-        np.testing.assert_allclose(host(lse), host(lse_ref), atol=2e-3, rtol=0)
+        assert _noalloc_c_abi(dims, cache, q, z, lse, splits) == 0
+        assert _noalloc_status() == 0
+        zh, lh = host(z), host(lse)
+        for b in range(wl.batch):
+            close(zh[b], ref[b][0], f"z seq {b}, call {call}")
+            np.testing.assert_allclose(lh[b], ref[b][1], atol=2e-3, rtol=0)
+        close(zh, host(z_ws), f"z vs workspace entry point, call {call}")
+        np.testing.assert_allclose(lh, host(lse_ws), atol=2e-3, rtol=0)
+
+
+def test_noalloc_reports_device_range_errors():
+    lens = np.array([100, 130])
+    wl = synth.reduced(synth.V2_BATCH64, "noalloc_bad", 53, 2, 0, 0, new_tokens=0)
+    pc = synth.make_paged_cache(wl, lens)
+    bt = pc.block_table.copy()
+    bt[1][1] = pc.num_pages + 3            # an out-of-range page entry
+    q_host = synth.make_q_lat(wl)
+    dims = lib_dims(wl)
+    cache = dev_cache(dataclasses.replace(pc, block_table=bt), lens)
+    z = torch.full((2, 128, 512), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(2, 128, dtype=torch.float32, device="cuda")
+    assert _noalloc_c_abi(dims, cache, dev(q_host, wl), z, lse) == 0
+    assert _noalloc_status() == 6          # MLA_ERR_DEVICE_RANGE
+    assert _noalloc_status() == 0          # reading clears it
+    zh, lh = host(z), host(lse)
+    assert np.all(zh[1] == 0) and np.all(np.isneginf(lh[1]))
+    zr, _ = oracle.attend_latent(q_host[0], pc.rows_f32(0, lens[0]), oracle_dims(wl))
+    assert_bf16_close(zh[0], zr, "seq 0")
 
 
 def test_noalloc_rejects_oversize_request():
@@ -87,7 +122,12 @@ def test_noalloc_rejects_oversize_request():
     cache = dev_cache(pc, lens)
     z = torch.full((2, 128, 512), 3.0, dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros(2, 128, dtype=torch.float32, device="cuda")
-    # 1000 partitions need ~500 MB of partials: beyond the fixed scratch
-    assert _noalloc_c_abi(dims, cache, q, z, lse, splits=1000) == 4   # MLA_ERR_WORKSPACE
+    # 31 partitions need 16 MiB of partials alone: beyond the fixed scratch;
+    # 1000 need ~500 MB
+    for splits in (31, 1000):
+        assert _noalloc_c_abi(dims, cache, q, z, lse, splits=splits) == 4   # MLA_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert torch.all(z == 3.0)   # nothing was enqueued
+    assert _noalloc_c_abi(dims, cache, q, z, lse, splits=30) == 0
+    assert _noalloc_status() == 0
+    torch.cuda.synchronize()
