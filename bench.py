@@ -47,6 +47,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MLA decode cached-token·heads/s and % of HBM / bf16 tensor-core roofline"
 UNIT = "cached-token·heads/s"
 ROW_BYTES = 576 * 2                 # one cached row: c (512) + k_R (64), bf16
+INT8_ROW_BYTES = 656                # int8 row: 512 codes, 64 bf16 k_R, scale, padding
 FLOP_PER_ROW_HEAD = 2 * 576 + 2 * 512
 
 # Launches of this library per decode step (checked against the ncu launch
@@ -89,9 +90,16 @@ def describe(wl):
     else:
         what = "full layer step: append + absorb_q (W_DQ) + attention + unabsorb (W_UV, W_O)"
         rows = f"cached rows {wl.prior_min}..{wl.prior_max} + {wl.new_tokens} new"
+    fmt = ("; int8 cache rows (codes x 2^e per row, k_R bf16, 656 B)" if wl.cache == "int8"
+           else "")
     return (f"{wl.name}: batch {wl.batch}/GPU, {wl.n_heads} heads, d_model {wl.d_model}, "
             f"q_lora {wl.d_q}, d_c {wl.d_c}, d_rope {wl.d_rope}, d_nope {wl.d_nope}, d_v {wl.d_v}, "
-            f"{rows}, {wl.page_size}-row pages{' (shuffled)' if wl.shuffle_pages else ''}; {what}")
+            f"{rows}, {wl.page_size}-row pages{' (shuffled)' if wl.shuffle_pages else ''}{fmt}; "
+            f"{what}")
+
+
+def row_bytes(wl):
+    return INT8_ROW_BYTES if wl.cache == "int8" else ROW_BYTES
 
 
 def attended_lengths(wl, prior):
@@ -103,7 +111,7 @@ def algorithmic(wl, lens):
     """Bytes / FLOPs that any implementation must move / do, per step and per attention call."""
     B, H = wl.batch, wl.n_heads
     rows = int(lens.sum())
-    attn_bytes = rows * ROW_BYTES + B * H * 576 * 2 + B * H * 512 * 2   # cache + q_lat + z
+    attn_bytes = rows * row_bytes(wl) + B * H * 576 * 2 + B * H * 512 * 2   # cache + q_lat + z
     attn_flops = rows * H * FLOP_PER_ROW_HEAD
     if attention_only(wl):
         return dict(rows=rows, attn_bytes=attn_bytes, attn_flops=attn_flops,
@@ -112,7 +120,7 @@ def algorithmic(wl, lens):
     params = (wl.d_c + wl.d_rope) * wl.d_model + (wl.d_q * wl.d_model if wl.d_q else 0) \
         + H * (wl.d_nope + wl.d_rope) * dq + H * wl.d_nope * wl.d_c + H * wl.d_v * wl.d_c \
         + wl.d_model * H * wl.d_v
-    step_bytes = attn_bytes + 2 * params + B * ROW_BYTES + 2 * B * wl.d_model * 2
+    step_bytes = attn_bytes + 2 * params + B * row_bytes(wl) + 2 * B * wl.d_model * 2
     step_flops = attn_flops + 2 * B * params
     return dict(rows=rows, attn_bytes=attn_bytes, attn_flops=attn_flops, step_bytes=step_bytes,
                 step_flops=step_flops, params=params)
@@ -246,12 +254,20 @@ def _oracle_dims(wl):
 
 def _oracle_unit(wl, W, pc, h, q):
     """f(b, n): the oracle's work for sequence b over its first n attended rows
-    (a whole un-absorbed decode step, or the latent attention alone)."""
+    (a whole un-absorbed decode step, or the latent attention alone); int8 rows
+    are read back through the oracle's dequantisation."""
     import oracle
     od = _oracle_dims(wl)
+
+    def rows(b, n):
+        if wl.cache != "int8":
+            return pc.rows_f32(b, n)
+        codes, exps, k_r = pc.fields(b, n)
+        return np.concatenate([oracle.dequantize_int8_pow2(codes, exps), k_r], axis=1)
+
     if attention_only(wl):
-        return lambda b, n: oracle.attend_latent(q[b], pc.rows_f32(b, n), od)
-    return lambda b, n: oracle.decode_step(h[b:b + 1], [pc.rows_f32(b, n - 1)], W, od)
+        return lambda b, n: oracle.attend_latent(q[b], rows(b, n), od)
+    return lambda b, n: oracle.decode_step(h[b:b + 1], [rows(b, n - 1)], W, od)
 
 
 def cpu_baseline_sample(wl, W, pc, h, q, lens, budget_s=20.0):
@@ -288,15 +304,20 @@ def run_mine(args):
     attn_only = attention_only(wl)
     prior = synth.make_prior_lengths(wl)
     lens = attended_lengths(wl, prior)
-    pc = synth.make_paged_cache(wl, prior)
+    int8 = wl.cache == "int8"
+    pc = synth.make_paged_cache_int8(wl, prior) if int8 else synth.make_paged_cache(wl, prior)
     W = None if attn_only else synth.make_weights(wl)
     h = None if attn_only else synth.make_hidden(wl)
     q = synth.make_q_lat(wl) if attn_only else None
     dims = L.Dims(wl.n_heads, wl.d_c, wl.d_rope, wl.d_nope, wl.d_v, wl.page_size, L.MLA_BF16,
-                  wl.rope_layout, wl.rope_base, wl.rms_eps)
+                  wl.rope_layout, wl.rope_base, wl.rms_eps,
+                  cache_format=L.MLA_CACHE_INT8 if int8 else L.MLA_CACHE_NATIVE)
     dev = torch.device("cuda", local)
     bf = lambda a: torch.from_numpy(a).to(dev).to(torch.bfloat16)
-    pool = torch.from_numpy(pc.pool.view(np.int16)).to(dev).view(torch.bfloat16)
+    if int8:
+        pool = torch.from_numpy(pc.pool).to(dev)
+    else:
+        pool = torch.from_numpy(pc.pool.view(np.int16)).to(dev).view(torch.bfloat16)
     cache = L.PagedCache(pool, torch.from_numpy(pc.block_table).to(dev),
                          torch.from_numpy(lens.astype(np.int32)).to(dev))
     stream = torch.cuda.current_stream()
@@ -444,7 +465,7 @@ def run_mine(args):
     h2d = sum(t.numel() * t.element_size() for t in inputs)
     d2h = output.numel() * output.element_size()
     l2 = ("no flush: per-step inputs (cache %.0f MB%s) exceed the 126 MB L2"
-          % (alg["rows"] * ROW_BYTES / 1e6,
+          % (alg["rows"] * row_bytes(wl) / 1e6,
              "" if attn_only else " + weights %.0f MB" % (2 * alg["params"] / 1e6)))
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -522,7 +543,8 @@ def run_reference(args):
     wl = workload(args.workload, 0)
     prior = synth.make_prior_lengths(wl)
     lens = attended_lengths(wl, prior)
-    pc = synth.make_paged_cache(wl, prior)
+    pc = (synth.make_paged_cache_int8(wl, prior) if wl.cache == "int8"
+          else synth.make_paged_cache(wl, prior))
     attn_only = attention_only(wl)
     W = None if attn_only else synth.make_weights(wl)
     h = None if attn_only else synth.make_hidden(wl)

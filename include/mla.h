@@ -74,6 +74,23 @@ typedef enum {
 enum { MLA_BF16 = 0, MLA_FP32 = 1 };
 enum { MLA_ROPE_INTERLEAVED = 0, MLA_ROPE_HALF = 1 };
 
+/* Cache row formats.
+ *   MLA_CACHE_NATIVE: a row is [c ; k_R] in dims->dtype (d_c + d_rope values).
+ *   MLA_CACHE_INT8 (MLA_BF16 only): the KV cache stored at lower precision
+ *     ("DeepSeek-V3多头潜在注意力(MLA)架构", 多头潜在注意力与KV缓存优化: INT8 or
+ *     INT4 keys and values).  A row is MLA_INT8_ROW_BYTES = 656 bytes:
+ *       bytes [0, 512)    c as int8 codes q_j in [-127, 127],
+ *       bytes [512, 640)  k_R as 64 bf16 values (not quantised),
+ *       bytes [640, 644)  the row's scale s = 2^e as an fp32 value,
+ *       bytes [644, 656)  zero.
+ *     The row holds c_j = q_j * s with e the smallest integer such that
+ *     max_j |c_j| <= 127 * 2^e, q_j = round-half-even(c_j / s).  Because s is a
+ *     power of two, q_j * s is exactly representable in bf16: decode attention
+ *     over an int8 cache computes exactly what it computes over the bf16 rows
+ *     [q * s ; k_R]. */
+enum { MLA_CACHE_NATIVE = 0, MLA_CACHE_INT8 = 1 };
+enum { MLA_INT8_ROW_BYTES = 656 };
+
 /* Sizes of one MLA layer.
  *   n_heads, d_nope (per-head content query/key width), d_v (per-head value
  *   width), d_c (latent width), d_rope (decoupled RoPE width, shared key).
@@ -88,12 +105,14 @@ typedef struct {
   int dtype;        /* MLA_BF16 | MLA_FP32 */
   int rope_layout;  /* MLA_ROPE_INTERLEAVED | MLA_ROPE_HALF */
   double rope_base, rms_eps, softmax_scale;
+  int cache_format; /* MLA_CACHE_NATIVE (0) | MLA_CACHE_INT8 */
 } mla_dims;
 
 /* The paged latent cache (device memory, caller-owned).
  *   pool: [num_pages][page_size][d_c + d_rope] elements of dims->dtype; a row is
  *         [c (d_c) ; k_R (d_rope)] ("从零理解 MLA", 解耦 RoPE absorbed_step caches
- *         cat([c_kv, k_r])).  Row s of sequence b lives at page
+ *         cat([c_kv, k_r])); with MLA_CACHE_INT8 a row is the 656-byte int8 row
+ *         described above, [num_pages][page_size][656] bytes.  Row s of sequence b lives at page
  *         block_table[b * max_pages_per_seq + s / page_size], slot s % page_size.
  *   seq_lens[b]: rows of sequence b that decode attention reads (rows
  *         0 .. seq_lens[b]-1).  mla_cache_append does not change it. */

@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(HERE, "libmla_b200.so")
 
 MLA_BF16, MLA_FP32 = 0, 1
 MLA_ROPE_INTERLEAVED, MLA_ROPE_HALF = 0, 1
+MLA_CACHE_NATIVE, MLA_CACHE_INT8 = 0, 1
+MLA_INT8_ROW_BYTES = 656
 
 STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
           3: "MLA_ERR_ALIGNMENT", 4: "MLA_ERR_WORKSPACE", 5: "MLA_ERR_CUDA",
@@ -43,7 +45,7 @@ class _Dims(ctypes.Structure):
                 ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int), ("page_size", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("rope_layout", ctypes.c_int),
                 ("rope_base", ctypes.c_double), ("rms_eps", ctypes.c_double),
-                ("softmax_scale", ctypes.c_double)]
+                ("softmax_scale", ctypes.c_double), ("cache_format", ctypes.c_int)]
 
 
 class _Cache(ctypes.Structure):
@@ -66,6 +68,7 @@ class Dims:
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
     softmax_scale: float = 0.0
+    cache_format: int = MLA_CACHE_NATIVE
 
     def c(self) -> _Dims:
         return _Dims(*dataclasses.astuple(self))

@@ -31,6 +31,9 @@ inline mla_status check_dims(const mla_dims *d) {
     return MLA_ERR_INVALID_ARG;
   if (!(d->rope_base > 0.0) || !(d->rms_eps >= 0.0) || !(d->softmax_scale >= 0.0))
     return MLA_ERR_INVALID_ARG;
+  if (d->cache_format != MLA_CACHE_NATIVE && d->cache_format != MLA_CACHE_INT8)
+    return MLA_ERR_INVALID_ARG;
+  if (d->cache_format == MLA_CACHE_INT8 && d->dtype != MLA_BF16) return MLA_ERR_UNSUPPORTED;
   if (d->dtype == MLA_FP32) {
     if (d->n_heads > 256 || d->d_c > 1024 || (d->d_c % 4) || d->d_nope > 256 || d->d_v > 256)
       return MLA_ERR_UNSUPPORTED;

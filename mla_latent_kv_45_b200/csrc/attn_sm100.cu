@@ -75,6 +75,7 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kWarpLoad = 8, kWarpS = 9, kWarpPV = 10, kWarpV = 11;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kI8Row = 656;      // bytes of an int8 cache row (512 codes, 64 bf16 k_R, scale, pad)
 constexpr uint32_t kSleepNs = 20000;   // suspend hint of a waiting thread (woken at completion)
 
 // Shared memory (byte offsets from a 1024-byte aligned base).  Every operand
@@ -113,7 +114,8 @@ constexpr uint32_t kIdescPV = idesc_bf16(256, 128, 1, 1);   // A = V^T, B = P (M
 constexpr uint16_t kBoth = 3;
 
 struct Bars {
-  uint64_t k_full[kKSlots];   // even CTA: both CTAs' row chunks landed (tx)
+  uint64_t k_full[kKSlots];   // even CTA: both CTAs' row chunks landed (tx; int8 rows: 2 arrivals)
+  uint64_t k_land[kKSlots];   // int8 rows: this CTA's chunk landed (local tx), before conversion
   uint64_t k_empty[kKSlots];  // the score MMAs reading the slot complete (pair commit)
   uint64_t v_land[kVSlots];   // this CTA's latent chunk landed (local tx)
   uint64_t v_full[kVSlots];   // even CTA: both CTAs' latent chunks ready (2 arrivals)
@@ -188,6 +190,34 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 16 int8 codes times the row's power-of-two scale s, as 16 bf16 values (two
+// 16-byte units, element order kept).  q + 128 is placed in the low mantissa
+// byte of 2^23, so fma(2^23 + q + 128, s, -(2^23 + 128) s) = q s exactly, and
+// q s (at most 8 significant bits) is exact in bf16.
+__device__ __forceinline__ void i8x16_to_bf16(const uint4 in, float s, uint4 &lo, uint4 &hi) {
+  const float bias = -8388736.0f * s;
+  const uint32_t w[4] = {in.x ^ 0x80808080u, in.y ^ 0x80808080u, in.z ^ 0x80808080u,
+                         in.w ^ 0x80808080u};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float f[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      f[k] = fmaf(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540u + k)), s, bias);
+    o[2 * i] = pack_bf16(f[0], f[1]);
+    o[2 * i + 1] = pack_bf16(f[2], f[3]);
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// The fp32 scale of an int8 row (bytes 640..643 of its 656).
+__device__ __forceinline__ float int8_row_scale(const AttnArgs &a, int page, int r) {
+  return __ldg(reinterpret_cast<const float *>(static_cast<const uint8_t *>(a.pool) +
+                                               ((long)page * kPage + r) * kI8Row + 640));
+}
 
 // Named barrier over the 256 softmax threads; the second form also returns
 // whether any of them passed true.
@@ -281,10 +311,21 @@ struct StepCursor {
   }
 };
 
+// kI8: the cache holds 656-byte int8 rows (MLA_CACHE_INT8).  tm_rows then maps
+// the rows' bf16 k_R columns, tm_i8k 64 int8 columns x 64 rows (score chunks)
+// and tm_i8v 128 int8 columns x 64 rows (latent columns for P.V); the int8
+// chunks land in the upper half of their ring slot and the loading warp turns
+// them in place into the same bf16 operand layout the bf16 rows arrive in.
+template <bool kI8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_rows,
-                      const __grid_constant__ CUtensorMap tm_q, const AttnArgs a,
+                      const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_i8k,
+                      const __grid_constant__ CUtensorMap tm_i8v, const AttnArgs a,
                       const float scale_log2) {
+#if MLA_ATTN_PREFETCH > 0
+  constexpr long kRowBytes = kI8 ? kI8Row : kRow * 2;
+#endif
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -298,7 +339,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kKSlots; ++s) {
-      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_full[s], kI8 ? 2 : 1);
+      mbar_init(&bars->k_land[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
     for (int s = 0; s < kVSlots; ++s) {
@@ -326,6 +368,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == kWarpLoad && lane == 0) {
     prefetch_tmap(&tm_rows);
     prefetch_tmap(&tm_q);
+    if (kI8) {
+      prefetch_tmap(&tm_i8k);
+      prefetch_tmap(&tm_i8v);
+    }
   }
   if (warp == kWarpS) {
     tmem_alloc_pair(&bars->tmem_base, kTmemCols);
@@ -344,7 +390,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   StepCursor cur;
   cur.init(a, hdr, part);
 
-  if (warp == kWarpLoad) {
+  if (kI8 && warp == kWarpLoad) {
+    // ---------- int8 rows: this CTA's 128 rows of each step, 64 columns a chunk,
+    // converted in place by the whole warp; the k_R chunk (bf16) is used as loaded
+    int nk = 0, pend_slot = 0, pend_nk = 0, pend_c = 0;
+    bool ok = true, pend = false, pend_has[2] = {false, false};
+    float pend_sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    // chunk idx (in `slot`) landed: int8 codes of page sp at +8 KB + 4 KB sp, row r
+    // at 64 r; bf16 out at +8 KB sp, row r at 128 r, 16-byte unit u at (u ^ (r & 7)) << 4.
+    // Page 1's output covers page 0's input and, from row 32 on, its own: page 0
+    // is converted first, and every 32-row batch is read before it is written.
+    auto finish_k = [&](int slot, int idx, int c, const bool (&has)[2],
+                        const float (&sc)[2][2]) -> bool {
+      if (!wait_bar(ctx, &bars->k_land[slot], (idx / kKSlots) & 1)) return false;
+      if (c < 8) {
+        uint8_t *base = smem + kOffK + slot * kKChunk;
+        for (int sp = 0; sp < 2; ++sp) {
+          if (!has[sp]) continue;
+          for (int hf = 0; hf < 2; ++hf) {
+            const int r = 32 * hf + lane;
+            const uint4 *in = reinterpret_cast<const uint4 *>(base + 8192 + 4096 * sp + 64 * r);
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = in[j];
+            __syncwarp();
+            uint8_t *out = base + kBox * sp + 128 * r;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 lo, hi;
+              i8x16_to_bf16(v[j], sc[sp][hf], lo, hi);
+              *reinterpret_cast<uint4 *>(out + (((2 * j) ^ (r & 7)) << 4)) = lo;
+              *reinterpret_cast<uint4 *>(out + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+            }
+            __syncwarp();
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(lead(&bars->k_full[slot]));
+      return true;
+    };
+    for (; cur.valid && ok; cur.advance(a)) {
+      const int np = cur.npages();
+      int pages[2];
+      bool has[2];
+      float sc[2][2];
+      for (int sp = 0; sp < 2; ++sp) {
+        const int j = 2 * (int)rank + sp;
+        pages[sp] = -1;
+        if (j < np) {
+          int page = cur.page(a, j);
+          if (page < 0 || page >= a.num_pages) {
+            if (lane == 0) {
+              set_error(a.err, kErrRange);
+              a.bad[cur.seg.b] = 1;
+            }
+            page = 0;
+          }
+          pages[sp] = page;
+        }
+        has[sp] = pages[sp] >= 0;
+        for (int hf = 0; hf < 2; ++hf)
+          sc[sp][hf] = has[sp] ? int8_row_scale(a, pages[sp], 32 * hf + lane) : 0.f;
+      }
+      const int nown = (int)has[0] + (int)has[1];
+      for (int c = 0; c < 9; ++c, ++nk) {
+        const int slot = nk % kKSlots;
+        if (nk >= kKSlots && !wait_bar(ctx, &bars->k_empty[slot], ((nk / kKSlots) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          uint8_t *dst = smem + kOffK + slot * kKChunk;
+          if (c < 8) {
+            mbar_expect_tx(&bars->k_land[slot], nown * 4096);
+            for (int sp = 0; sp < 2; ++sp)
+              if (has[sp])
+                tma_load_2d_hint(dst + 8192 + 4096 * sp, &tm_i8k, 64 * c, pages[sp] * kPage,
+                                 &bars->k_land[slot], l2_policy_evict_last());
+          } else {
+            mbar_expect_tx(&bars->k_land[slot], nown * kBox);
+            for (int sp = 0; sp < 2; ++sp)
+              if (has[sp])
+                tma_load_2d_hint(dst + kBox * sp, &tm_rows, 512, pages[sp] * kPage,
+                                 &bars->k_land[slot], l2_policy_evict_last());
+          }
+        }
+        __syncwarp();
+        if (pend && !finish_k(pend_slot, pend_nk, pend_c, pend_has, pend_sc)) {
+          ok = false;
+          break;
+        }
+        pend = true;
+        pend_slot = slot;
+        pend_nk = nk;
+        pend_c = c;
+        for (int sp = 0; sp < 2; ++sp) {
+          pend_has[sp] = has[sp];
+          pend_sc[sp][0] = sc[sp][0];
+          pend_sc[sp][1] = sc[sp][1];
+        }
+      }
+    }
+    if (ok && pend) finish_k(pend_slot, pend_nk, pend_c, pend_has, pend_sc);
+  } else if (warp == kWarpLoad) {
     // ------------------------- this CTA's 128 rows of each step, in 64-column chunks
     if (lane == 0) {
       int nk = 0;
@@ -359,8 +509,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (j < ahead.npages()) {
             const int page = ahead.page(a, j);
             if (page >= 0 && page < a.num_pages)
-              prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRow * 2,
-                          kPage * kRow * 2);
+              prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRowBytes,
+                          kPage * kRowBytes);
           }
         }
         ahead.advance(a);
@@ -374,8 +524,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (j < ahead.npages()) {
               const int page = ahead.page(a, j);
               if (page >= 0 && page < a.num_pages)
-                prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRow * 2,
-                            kPage * kRow * 2);
+                prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRowBytes,
+                            kPage * kRowBytes);
             }
           }
           ahead.advance(a);
@@ -416,12 +566,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpV) {
     // ------------- each page's 64 rows of this CTA's 256 latent columns (P.V A operand)
     int nv = 0, prev_slot = 0, prev_valid = kPage;
+    float prev_sc0 = 0.f, prev_sc1 = 0.f;
     bool ok = true, pending = false;
     // hands chunk `idx` (landed) to the P.V issuer; rows past the sequence end
     // hold arbitrary bytes and are zeroed so that 0 * (stale bytes) cannot reach O
-    auto finish = [&](int slot, int idx, int valid) -> bool {
+    auto finish = [&](int slot, int idx, int valid, float sc0, float sc1) -> bool {
       if (!wait_bar(ctx, &bars->v_land[slot], (idx / kVSlots) & 1)) return false;
-      if (valid < kPage) {
+      if (kI8) {
+        // int8 codes of row r at +8 KB + 128 r (128 latent columns) -> bf16 boxes
+        // 0 (columns 0-63) at 128 r and 1 (64-127) at 8 KB + 128 r: box 1's row r is
+        // exactly the input row r, which the lane has read before it writes
+        uint8_t *dst = smem + kOffV + slot * kVChunk;
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = 32 * hf + lane;
+          const float sc = hf ? sc1 : sc0;
+          uint4 v[8];
+          const uint4 *in = reinterpret_cast<const uint4 *>(dst + kBox + 128 * r);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = in[j];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+            if (r < valid) i8x16_to_bf16(v[j], sc, lo, hi);
+            uint8_t *out = dst + (j >> 2) * kBox + 128 * r;
+            const int u = 2 * (j & 3);
+            *reinterpret_cast<uint4 *>(out + ((u ^ (r & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4 *>(out + (((u + 1) ^ (r & 7)) << 4)) = hi;
+          }
+        }
+        fence_proxy_async_smem();
+      } else if (valid < kPage) {
         uint8_t *dst = smem + kOffV + slot * kVChunk;
         for (int i = lane; i < (kPage - valid) * 16; i += 32) {
           const int row = valid + (i >> 4), box = (i >> 3) & 1, piece = i & 7;
@@ -448,25 +622,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (lane == 0) {
             uint8_t *dst = smem + kOffV + slot * kVChunk;
-            mbar_expect_tx(&bars->v_land[slot], kVChunk);
-            // box sub: latent columns 256 blk + 128 r + 64 sub, all 64 rows; the last
-            // read of these bytes, so evict-first
-            for (int sub = 0; sub < 2; ++sub)
-              tma_load_2d_hint(dst + sub * kBox, &tm_rows, 256 * blk + 128 * (int)rank + 64 * sub,
-                               page * kPage, &bars->v_land[slot], l2_policy_evict_first());
+            // the last read of these bytes, so evict-first
+            if (kI8) {
+              // int8 latent columns 256 blk + 128 r .. +128 of all 64 rows, upper half
+              mbar_expect_tx(&bars->v_land[slot], kBox);
+              tma_load_2d_hint(dst + kBox, &tm_i8v, 256 * blk + 128 * (int)rank, page * kPage,
+                               &bars->v_land[slot], l2_policy_evict_first());
+            } else {
+              // box sub: latent columns 256 blk + 128 r + 64 sub, all 64 rows
+              mbar_expect_tx(&bars->v_land[slot], kVChunk);
+              for (int sub = 0; sub < 2; ++sub)
+                tma_load_2d_hint(dst + sub * kBox, &tm_rows,
+                                 256 * blk + 128 * (int)rank + 64 * sub, page * kPage,
+                                 &bars->v_land[slot], l2_policy_evict_first());
+            }
+          }
+          float sc0 = 0.f, sc1 = 0.f;
+          if (kI8) {
+            sc0 = int8_row_scale(a, page, lane);
+            sc1 = int8_row_scale(a, page, lane + 32);
           }
           __syncwarp();
-          if (pending && !finish(prev_slot, nv - 1, prev_valid)) {
+          if (pending && !finish(prev_slot, nv - 1, prev_valid, prev_sc0, prev_sc1)) {
             ok = false;
             break;
           }
           prev_slot = slot;
           prev_valid = valid;
+          prev_sc0 = sc0;
+          prev_sc1 = sc1;
           pending = true;
         }
       }
     }
-    if (ok && pending) finish(prev_slot, nv - 1, prev_valid);
+    if (ok && pending) finish(prev_slot, nv - 1, prev_valid, prev_sc0, prev_sc1);
   } else if (warp == kWarpS) {
     // ----------------- q_lat halves (both CTAs); the even CTA issues the score MMAs
     if (lane == 0) {
@@ -809,24 +998,55 @@ bool make_map(CUtensorMap *m, const void *base, long rows, int box_cols, int box
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D byte map over int8 rows (656 bytes each); box = box_bytes x box_rows.
+bool make_map_i8(CUtensorMap *m, const void *base, long rows, int box_bytes, int box_rows,
+                 CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kI8Row, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kI8Row};
+  const cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool kI8>
+cudaError_t launch_attn_t(const AttnArgs &a, int parts, cudaStream_t s) {
+  static api::PerDeviceOnce smem_attr;
+  cudaError_t e = smem_attr.run([] {
+    return cudaFuncSetAttribute(attn_sm100_kernel<kI8>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  });
+  if (e != cudaSuccess) return e;
+  CUtensorMap tm_rows, tm_q, tm_i8k, tm_i8v;
+  const long pool_rows = (long)a.num_pages * kPage;
+  const long q_rows = (long)a.batch * kHeads;
+  if (!make_map(&tm_q, a.q_lat, q_rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (kI8) {
+    // k_R (bytes 512..639) as swizzled bf16 boxes; the codes in plain boxes that
+    // the kernel converts
+    if (!make_map_i8(&tm_rows, a.pool, pool_rows, 128, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_i8(&tm_i8k, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_i8(&tm_i8v, a.pool, pool_rows, 128, kPage, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tm_rows, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    tm_i8k = tm_rows;
+    tm_i8v = tm_rows;
+  }
+  const float scale_log2 = a.scale * 1.4426950408889634f;
+  return launch_pdl(attn_sm100_kernel<kI8>, dim3(2 * parts), dim3(kThreads), kSmemBytes, s,
+                    tm_rows, tm_q, tm_i8k, tm_i8v, a, scale_log2);
+}
+
 }  // namespace
 
 cudaError_t launch_attn(const AttnArgs &a, int parts, cudaStream_t s) {
-  static api::PerDeviceOnce smem_attr;
-  cudaError_t e = smem_attr.run([] {
-    return cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kSmemBytes);
-  });
-  if (e != cudaSuccess) return e;
-  CUtensorMap tm_rows, tm_q;
-  const long pool_rows = (long)a.num_pages * kPage;
-  const long q_rows = (long)a.batch * kHeads;
-  if (!make_map(&tm_rows, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&tm_q, a.q_lat, q_rows, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  const float scale_log2 = a.scale * 1.4426950408889634f;
-  return launch_pdl(attn_sm100_kernel, dim3(2 * parts), dim3(kThreads), kSmemBytes, s, tm_rows,
-                    tm_q, a, scale_log2);
+  return a.int8_rows ? launch_attn_t<true>(a, parts, s) : launch_attn_t<false>(a, parts, s);
 }
 
 }  // namespace sm100

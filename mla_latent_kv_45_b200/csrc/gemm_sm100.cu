@@ -22,6 +22,8 @@
 // warps 2-5 epilogue.  Every wait is bounded (globaltimer).
 #include <cuda.h>
 
+#include <mutex>
+
 #include "api_checks.h"
 #include "ptx.cuh"
 #include "sm100.h"
@@ -377,10 +379,66 @@ int gemm_splits(int m_tiles, int heads, int k_chunks) {
   return (k_chunks + per - 1) / per;
 }
 
+namespace {
+
+cudaError_t set_smem_attr() {
+  static api::PerDeviceOnce smem_attr;
+  return smem_attr.run([] {
+    return cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                232448);
+  });
+}
+
+// Clusters of `size` CTAs (two CTAs' worth of shared memory per SM) that the
+// device can hold at once, or 0 if that cannot be determined (queried once per
+// device and size).
+int max_active_clusters(int size) {
+  static std::mutex lock;
+  static int known[64][kMaxClusterSplits + 1];
+  static bool init = false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || size < 1 ||
+      size > kMaxClusterSplits)
+    return 0;
+  {
+    std::lock_guard<std::mutex> g(lock);
+    if (!init) {
+      for (auto &row : known)
+        for (int &v : row) v = -1;
+      init = true;
+    }
+    if (known[dev][size] >= 0) return known[dev][size];
+  }
+  if (set_smem_attr() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(size);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 232448 / 2 - 256;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = size;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_sm100_kernel, &cfg) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> g(lock);
+  known[dev][size] = n;
+  return n;
+}
+
+}  // namespace
+
 int gemm_cluster_splits(int m_tiles, int heads, int k_chunks) {
-  const int s = gemm_splits(m_tiles, heads, k_chunks);
-  if (s <= kMaxClusterSplits) return s;
-  const int per = (k_chunks + kMaxClusterSplits - 1) / kMaxClusterSplits;
+  int s = gemm_splits(m_tiles, heads, k_chunks);
+  if (s > kMaxClusterSplits) s = kMaxClusterSplits;
+  // one cluster per tile: take the largest split whose clusters all fit on the
+  // device at once (clusters live inside one GPC, so a size that packs badly
+  // would leave some tiles for a second wave)
+  const int tiles = m_tiles * heads;
+  while (s > 2 && max_active_clusters(s) < tiles) --s;
+  const int per = (k_chunks + s - 1) / s;
   return (k_chunks + per - 1) / per;
 }
 
@@ -401,11 +459,7 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
       return cudaErrorInvalidValue;
   }
   const int n_step = cluster ? 128 : 256;
-  static api::PerDeviceOnce smem_attr;
-  cudaError_t ea = smem_attr.run([] {
-    return cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                232448);
-  });
+  const cudaError_t ea = set_smem_attr();
   if (ea != cudaSuccess) return ea;
   for (int n0 = 0; n0 < n; n0 += n_step) {
     const int nn = n - n0 < n_step ? n - n0 : n_step;

@@ -32,6 +32,13 @@ cudaError_t launch_append_finish(const float *xkv, int splits, int batch, int d_
                                  const int32_t *block_table, int max_pages, int *err,
                                  cudaStream_t s);
 
+// The same append into a 656-byte int8 row (MLA_CACHE_INT8, d_c = 512, d_rope = 64).
+cudaError_t launch_append_finish_int8(const float *xkv, int batch, int d_c, const RopeParams &rp,
+                                      const __nv_bfloat16 *gamma, float eps,
+                                      const int32_t *positions, uint8_t *pool, int num_pages,
+                                      int page_size, const int32_t *block_table, int max_pages,
+                                      int *err, cudaStream_t s);
+
 template <class T>
 cudaError_t launch_rope_q(const float *qr, int batch, int n_heads, int d_c, const RopeParams &rp,
                           const int32_t *positions, T *q_lat, cudaStream_t s);
@@ -70,6 +77,7 @@ struct AttnArgs {
   // Partial-softmax output (nullptr for z / lse): unnormalised O [batch][n_heads][d_c],
   // m (natural-log max) and l [batch][n_heads], fp32.
   float *pout_O, *pout_m, *pout_l;
+  int int8_rows;  // the pool holds 656-byte int8 rows (MLA_CACHE_INT8)
 };
 
 template <class T>

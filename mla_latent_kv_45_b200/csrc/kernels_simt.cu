@@ -164,6 +164,97 @@ template cudaError_t launch_append_finish<__nv_bfloat16>(
     const float *, int, int, int, const RopeParams &, const __nv_bfloat16 *, float,
     const int32_t *, __nv_bfloat16 *, int, int, const int32_t *, int, int *, cudaStream_t);
 
+// Cache append into an int8 row (656 bytes: 512 int8 codes, 64 bf16 k_R, the
+// fp32 scale 2^e, zero padding).  c = gamma * x / rms(x) is formed in fp32 as in
+// append_finish, then quantised with the row's power-of-two scale: e is the
+// smallest integer with max|c| <= 127 * 2^e and q = round-half-even(c / 2^e).
+__global__ void append_finish_int8(const float *xkv, int batch, int d_c, RopeParams rp,
+                                   const __nv_bfloat16 *gamma, float eps,
+                                   const int32_t *positions, uint8_t *pool, int num_pages,
+                                   int page_size, const int32_t *block_table, int max_pages,
+                                   int *err) {
+  extern __shared__ float x[];   // [d_c + d_rope]
+  __shared__ float red[32];
+  __shared__ float inv_rms, amax_s;
+  grid_dep_wait();
+  const int b = blockIdx.x;
+  const int row = d_c + rp.d_rope;
+  for (int i = threadIdx.x; i < row; i += blockDim.x) x[i] = xkv[(long)b * row + i];
+  __syncthreads();
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) ss += x[i] * x[i];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) inv_rms = 1.0f / sqrtf(v / (float)d_c + eps);
+  }
+  __syncthreads();
+  // c in fp32 (kept in place of x), then its largest magnitude
+  float am = 0.f;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) {
+    const float c = __bfloat162float(gamma[i]) * (x[i] * inv_rms);
+    x[i] = c;
+    am = fmaxf(am, fabsf(c));
+  }
+  am = warp_max(am);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) amax_s = v;
+  }
+  __syncthreads();
+  const float amax = amax_s;
+  // amax in [2^k, 2^(k+1)): 127 * 2^(k-6) = 1.98 * 2^k, so e is k - 6 or k - 5
+  int e = 0;
+  if (amax > 0.f) {
+    e = ilogbf(amax) - 6;
+    if (amax > ldexpf(127.f, e)) ++e;
+  }
+  const float inv_s = ldexpf(1.f, -e);
+  const int pos = positions[b];
+  const long cap = (long)max_pages * page_size;
+  int page = -1;
+  if (pos >= 0 && pos < cap) page = block_table[(long)b * max_pages + pos / page_size];
+  if (page < 0 || page >= num_pages) {
+    if (threadIdx.x == 0) set_error(err, kErrRange);
+    return;
+  }
+  uint8_t *dst = pool + ((long)page * page_size + pos % page_size) * 656;
+  for (int i = threadIdx.x; i < d_c; i += blockDim.x) {
+    const int q = max(-127, min(127, __float2int_rn(x[i] * inv_s)));
+    dst[i] = static_cast<uint8_t>(static_cast<int8_t>(q));
+  }
+  __nv_bfloat16 *kr = reinterpret_cast<__nv_bfloat16 *>(dst + d_c);
+  for (int i = threadIdx.x; i < rp.d_rope / 2; i += blockDim.x) {
+    int j0, j1;
+    rope_idx(rp, i, j0, j1);
+    float x0 = x[d_c + j0], x1 = x[d_c + j1];
+    rope_pair(rp, i, pos, x0, x1);
+    kr[j0] = __float2bfloat16_rn(x0);
+    kr[j1] = __float2bfloat16_rn(x1);
+  }
+  if (threadIdx.x < 4) {
+    uint32_t *tail = reinterpret_cast<uint32_t *>(dst + d_c + 2 * rp.d_rope);   // bytes 640..655
+    tail[threadIdx.x] = threadIdx.x == 0 ? __float_as_uint(ldexpf(1.f, e)) : 0u;
+  }
+}
+
+cudaError_t launch_append_finish_int8(const float *xkv, int batch, int d_c, const RopeParams &rp,
+                                      const __nv_bfloat16 *gamma, float eps,
+                                      const int32_t *positions, uint8_t *pool, int num_pages,
+                                      int page_size, const int32_t *block_table, int max_pages,
+                                      int *err, cudaStream_t s) {
+  const size_t smem = (d_c + rp.d_rope) * sizeof(float);
+  return launch_pdl(append_finish_int8, dim3(batch), dim3(256), smem, s, xkv, batch, d_c, rp,
+                    gamma, eps, positions, pool, num_pages, page_size, block_table, max_pages, err);
+}
+
 // ---------------------------------------------------------------------------
 // q_R = RoPE_pos(W_QR c_Q) written into the tail of each q_lat row
 // ---------------------------------------------------------------------------

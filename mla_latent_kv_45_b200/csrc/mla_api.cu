@@ -154,6 +154,7 @@ mla_status decode_attn_impl(const mla_dims *dims, const mla_paged_cache *cache, 
   a.part_m = reinterpret_cast<float *>(at(ws, L.part_m));
   a.part_l = reinterpret_cast<float *>(at(ws, L.part_l));
   a.err = pa.err;
+  a.int8_rows = d.cache_format == MLA_CACHE_INT8;
   a.pout_O = pO;
   a.pout_m = pm;
   a.pout_l = pl;
@@ -215,6 +216,11 @@ mla_status mla_cache_append(const mla_dims *dims, const mla_paged_cache *cache, 
   MLA_TRY(cuda_ok(sm100::append_proj(static_cast<const bf16 *>(h), static_cast<const bf16 *>(W_DKV),
                                      static_cast<const bf16 *>(W_KR), batch, d_model, xkv, err,
                                      s)));
+  if (d.cache_format == MLA_CACHE_INT8)
+    return cuda_ok(launch_append_finish_int8(
+        xkv, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
+        static_cast<uint8_t *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,
+        cache->max_pages_per_seq, err, s));
   return cuda_ok(launch_append_finish<bf16>(
       xkv, 1, batch, d.d_c, rp, static_cast<const bf16 *>(gamma), (float)d.rms_eps, positions,
       static_cast<bf16 *>(cache->pool), cache->num_pages, d.page_size, cache->block_table,

@@ -151,6 +151,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
   a.part_m = reinterpret_cast<float *>(ws + R.part_m);
   a.part_l = reinterpret_cast<float *>(ws + R.part_l);
   a.err = pa.err;
+  a.int8_rows = d.cache_format == MLA_CACHE_INT8;
   cudaError_t e;
   if (d.dtype == MLA_FP32) {
     e = launch_attn_simt<float>(a, parts, s);

@@ -17,6 +17,7 @@ Workloads (DeepSeek-V2 attention sizes from "从零理解 MLA", 实际配置:
 * ``v2_long``    bf16, batch 8, 131072 rows per sequence (positions 0..131071,
              the query's own row included), attention only.
 * ``v2_step128`` bf16, batch 128, 2048 cached rows + 1 new, whole layer step.
+* ``v2_batch64_int8``  ``v2_batch64`` over 656-byte int8 cache rows.
 
 Distributions: weights N(0, 0.02^2), hidden states N(0, 1), RMSNorm gain 1
 (optionally 1 + 0.1 N(0,1)), cached rows N(0, 1) (the scale of an
@@ -81,6 +82,7 @@ class Workload:
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
     rope_layout: int = 0     # 0 interleaved, 1 half-split
+    cache: str = "native"    # "native": rows in `dtype`; "int8": 656-byte int8 rows
 
     @property
     def row(self) -> int:
@@ -93,8 +95,11 @@ V2_BATCH64 = Workload("v2_batch64", 2, 64, 128, 5120, 1536, 512, 128, 64, 128, 6
 V2_LONG = Workload("v2_long", 3, 8, 128, 5120, 1536, 512, 128, 64, 128, 64, "bf16", 131072, 131072,
                    new_tokens=0)
 V2_STEP128 = Workload("v2_step128", 4, 128, 128, 5120, 1536, 512, 128, 64, 128, 64, "bf16", 2048, 2048)
+# the batch-64 workload (same seeds) over an int8 latent cache
+V2_BATCH64_INT8 = dataclasses.replace(V2_BATCH64, name="v2_batch64_int8", cache="int8")
 
-WORKLOADS = {w.name: w for w in (TINY, V2_SINGLE, V2_BATCH64, V2_LONG, V2_STEP128)}
+WORKLOADS = {w.name: w for w in (TINY, V2_SINGLE, V2_BATCH64, V2_LONG, V2_STEP128,
+                                 V2_BATCH64_INT8)}
 
 
 def reduced(base: Workload, name: str, wid: int, batch: int, prior_min: int, prior_max: int,
@@ -217,6 +222,72 @@ def make_paged_cache(wl: Workload, prior_lens: Optional[np.ndarray] = None,
             idx = np.arange(L)
             pool[bt[b][idx // ps], idx % ps] = vals
     return PagedCache(pool, bt, np.asarray(prior_lens, dtype=np.int64), ps)
+
+
+INT8_ROW_BYTES = 656
+
+
+@dataclasses.dataclass
+class Int8PagedCache:
+    """A paged pool of 656-byte int8 rows and its page table, as host arrays.
+
+    Row layout (the library's MLA_CACHE_INT8 format): bytes [0, 512) int8 codes
+    of c, [512, 640) k_R as 64 bf16 values, [640, 644) the row's scale 2^e as
+    an fp32 value, [644, 656) zero.  ``fields`` unpacks a sequence's rows
+    exactly (codes, exponents, k_R); turning them into values is the method's
+    arithmetic and left to the caller.
+    """
+    pool: np.ndarray          # [num_pages, page_size, 656] uint8
+    block_table: np.ndarray
+    prior_lens: np.ndarray
+    page_size: int
+
+    @property
+    def num_pages(self) -> int:
+        return self.pool.shape[0]
+
+    def raw_rows(self, b: int, length: int) -> np.ndarray:
+        idx = np.arange(length)
+        return self.pool[self.block_table[b][idx // self.page_size], idx % self.page_size]
+
+    def fields(self, b: int, length: int):
+        r = self.raw_rows(b, length)
+        codes = r[:, :512].view(np.int8).astype(np.int64)
+        k_r = bf16_to_f32(np.ascontiguousarray(r[:, 512:640]).view(np.uint16))
+        scale = np.ascontiguousarray(r[:, 640:644]).view(np.float32)[:, 0]
+        exps = np.round(np.log2(scale)).astype(np.int64)
+        return codes, exps, k_r
+
+
+def make_paged_cache_int8(wl: Workload, prior_lens: Optional[np.ndarray] = None,
+                          spare_pages: int = 0) -> Int8PagedCache:
+    """Pool of int8 rows with the same page assignment as ``make_paged_cache``.
+
+    Codes are round(32 N(0, 1)) clipped to [-127, 127], exponents uniform in
+    [-9, -4] (so values q 2^e have roughly the spread of an RMS-normalised
+    latent), k_R ~ N(0, 1) rounded to bf16.  Unfilled rows are zero bytes.
+    """
+    if prior_lens is None:
+        prior_lens = make_prior_lengths(wl)
+    ref = make_paged_cache(dataclasses.replace(wl, dtype="bf16"), prior_lens, spare_pages,
+                           fill=False)
+    pool = np.zeros(ref.pool.shape[:2] + (INT8_ROW_BYTES,), dtype=np.uint8)
+    g = rng(1000 * wl.wid + 16)
+    ps = wl.page_size
+    for b in range(wl.batch):
+        L = int(prior_lens[b])
+        if L == 0:
+            continue
+        codes = np.clip(np.round(32.0 * g.standard_normal((L, 512))), -127, 127).astype(np.int8)
+        exps = g.integers(-9, -3, size=L)
+        k_r = bf16_bits(g.standard_normal((L, 64), dtype=np.float32))
+        rows = np.zeros((L, INT8_ROW_BYTES), dtype=np.uint8)
+        rows[:, :512] = codes.view(np.uint8)
+        rows[:, 512:640] = k_r.view(np.uint8).reshape(L, 128)
+        rows[:, 640:644] = np.exp2(exps).astype(np.float32).view(np.uint8).reshape(L, 4)
+        idx = np.arange(L)
+        pool[ref.block_table[b][idx // ps], idx % ps] = rows
+    return Int8PagedCache(pool, ref.block_table, ref.prior_lens, ps)
 
 
 def make_q_lat(wl: Workload, tid: int = 14) -> np.ndarray:

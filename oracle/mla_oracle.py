@@ -29,6 +29,9 @@ Pins (tests/test_oracle_pins.py) -- every function below is pinned:
 * ``forward_naive``   causal brute force; equals the step-by-step absorbed loop.
 * ``gather_rows``     rows scattered one by one into a shuffled pool by the
                       layout's definition come back in logical order.
+* ``quantize_int8_pow2`` / ``dequantize_int8_pow2``  closed forms (code range,
+                      tightest scale, error <= s / 2), brute-force search of the
+                      exponent, half-to-even ties, torch.round on c / s.
 """
 
 from __future__ import annotations
@@ -46,6 +49,7 @@ __all__ = [
     "rms_norm", "latent_row", "queries", "absorb_q", "attend_latent",
     "attend_unabsorbed", "split_partial", "combine_splits", "unabsorb",
     "decode_step", "forward_naive", "absorbed_decode_loop", "gather_rows",
+    "INT8_MAX", "quantize_int8_pow2", "dequantize_int8_pow2",
 ]
 
 
@@ -183,6 +187,41 @@ def latent_row(h, W_DKV, W_KR, gamma, pos, dims: Dims) -> np.ndarray:
     c = rms_norm(x, gamma, dims.rms_eps)
     k = rope(h @ _f64(W_KR).T, _f64(pos), dims.rope_base, dims.rope_layout)
     return np.concatenate([c, k], axis=-1)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit latent rows: c as int8 codes times a power-of-two scale
+# ---------------------------------------------------------------------------
+
+INT8_MAX = 127
+
+
+def quantize_int8_pow2(c):
+    """Per-row int8 quantisation with a power-of-two scale.
+
+    "DeepSeek-V3多头潜在注意力(MLA)架构", 多头潜在注意力与KV缓存优化: the KV
+    cache may be stored at lower precision (INT8 or INT4), at some cost in
+    accuracy.  Reading taken here: each cached latent row c (d_c values) is
+    stored as int8 codes q and one scale s = 2**e, the smallest power of two
+    with max|c| / s <= 127, q = round-half-even(c / s); the row then reads back
+    as q * s.  (A power-of-two scale keeps c / s and q * s exact, at the cost of
+    at most one bit of the code range.)  An all-zero row gets e = 0.
+
+    ``c [..., d_c]`` -> ``q [..., d_c]`` (int64 codes in [-127, 127]), ``e [...]``.
+    """
+    c = _f64(c)
+    amax = np.abs(c).max(axis=-1)
+    e = np.zeros(amax.shape, dtype=np.int64)
+    nz = amax > 0
+    e[nz] = np.ceil(np.log2(amax[nz] / INT8_MAX)).astype(np.int64)
+    s = np.exp2(e.astype(np.float64))[..., None]
+    q = np.round(c / s)           # numpy rounds half to even
+    return q.astype(np.int64), e
+
+
+def dequantize_int8_pow2(q, e):
+    """q * 2**e: the latent values an int8 row holds."""
+    return _f64(q) * np.exp2(_f64(e))[..., None]
 
 
 # ---------------------------------------------------------------------------

@@ -34,6 +34,19 @@ def test_header_symbols_exported(lib):
     assert set(syms) == set(L.EXPORTS)
 
 
+def test_split_kv_host_checks(lib):
+    d = V2.c()
+    c = _cache()
+    p = lib.mla_decode_attn_partial
+    assert p(ctypes.byref(d), ctypes.byref(c), 2, A, A, A, None, 0, A, 1 << 30, None) == 1
+    assert p(ctypes.byref(d), ctypes.byref(c), 2, A, A + 8, A, A, 0, A, 1 << 30, None) == 3
+    assert p(ctypes.byref(d), ctypes.byref(c), 2, A, A, A, A, 0, A, 100, None) == 4
+    m = lib.mla_merge_partials
+    assert m(ctypes.byref(d), 2, 0, A, A, A, A, None, None) == 1       # no parts
+    assert m(ctypes.byref(d), 2, 3, A + 4, A, A, A, None, None) == 3   # O misaligned
+    assert m(ctypes.byref(d), 2, 3, A, A, A, None, None, None) == 1    # null z
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert L.status_string(code)
@@ -79,6 +92,11 @@ def test_decode_attn_host_checks(lib):
     assert attn(lib, V2, _cache(), ws=None) == 1
     t = L.Dims(4, 16, 8, 8, 8, 16, 7)                        # bad dtype enum
     assert attn(lib, t, _cache()) == 1
+    i8 = L.Dims(128, 512, 64, 128, 128, 64, L.MLA_BF16, cache_format=L.MLA_CACHE_INT8)
+    assert attn(lib, i8, _cache(), wsb=100) == 4             # int8 rows accepted (bf16 sizes)
+    assert attn(lib, L.Dims(4, 16, 8, 8, 8, 16, L.MLA_FP32, cache_format=L.MLA_CACHE_INT8),
+                _cache()) == 2                               # int8 rows need the bf16 path
+    assert attn(lib, L.Dims(128, 512, 64, 128, 128, 64, cache_format=5), _cache()) == 1
 
 
 def test_append_absorb_unabsorb_host_checks(lib):

@@ -520,3 +520,58 @@ def test_pins_catch_gather_mistakes():
 
     for bad in (slot_swapped, pool_order):
         assert _fails(check_gather, bad)
+
+
+# ---------------------------------------------------------------------------
+# int8 latent rows (KV-cache quantisation, "DeepSeek-V3多头潜在注意力(MLA)架构",
+# 多头潜在注意力与KV缓存优化): codes times a power-of-two scale
+# ---------------------------------------------------------------------------
+
+def check_int8(quant, dequant):
+    rng = _r(91)
+    c = rng.standard_normal((40, 512)) * np.exp2(rng.integers(-12, 12, size=(40, 1)))
+    c[3] = 0.0
+    q, e = quant(c)
+    assert q.shape == c.shape and e.shape == (40,)
+    assert np.all(np.abs(q) <= 127)
+    s = np.exp2(e.astype(float))[:, None]
+    # the tightest power of two: the largest code uses more than half the range
+    nz = np.abs(c).max(1) > 0
+    assert np.all(np.abs(q[nz]).max(1) >= 64)
+    assert e[3] == 0 and np.all(q[3] == 0)
+    # brute force over exponents: the smallest e with max|round(c / 2^e)| <= 127
+    for i in np.flatnonzero(nz)[:8]:
+        best = min(k for k in range(-40, 40)
+                   if np.abs(np.round(c[i] / 2.0 ** k)).max() <= 127)
+        assert e[i] == best
+    # library rounding (half to even) of the scaled row, and the error bound
+    assert np.array_equal(q, torch.round(torch.from_numpy(c / s)).numpy().astype(np.int64))
+    d = dequant(q, e)
+    assert np.all(np.abs(d - c) <= s / 2)
+    # exact ties go to even codes
+    t = np.array([[0.5, 1.5, 2.5, -0.5, -2.5, 127.0]])
+    qt, et = quant(t)
+    assert et[0] == 0 and qt[0].tolist() == [0, 2, 2, 0, -2, 127]
+
+
+def test_int8_pins():
+    check_int8(oracle.quantize_int8_pow2, oracle.dequantize_int8_pow2)
+
+
+def test_pins_catch_int8_mistakes():
+    def loose_scale(c):      # scale one power of two too large
+        q, e = oracle.quantize_int8_pow2(c)
+        e = e + 1
+        return np.round(c / np.exp2(e.astype(float))[:, None]).astype(np.int64), e
+
+    def truncating(c):       # rounds toward zero
+        q, e = oracle.quantize_int8_pow2(c)
+        return np.trunc(c / np.exp2(e.astype(float))[:, None]).astype(np.int64), e
+
+    def half_up(c):          # rounds halves away from zero
+        q, e = oracle.quantize_int8_pow2(c)
+        x = c / np.exp2(e.astype(float))[:, None]
+        return (np.sign(x) * np.floor(np.abs(x) + 0.5)).astype(np.int64), e
+
+    for bad in (loose_scale, truncating, half_up):
+        assert _fails(check_int8, bad, oracle.dequantize_int8_pow2)

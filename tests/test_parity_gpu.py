@@ -361,7 +361,7 @@ def _set_rows(pc, b, rows):
 
 
 def _ramp_case():
-    """k_R of row s grows from x1 to x16 along each sequence, c stays N(0, 1):
+    """k_R of row s grows from x1 to x32 along each sequence, c stays N(0, 1):
     the position score, and with it each head's running maximum, rises step
     after step by far more than 2^8, while z stays a mean of N(0, 1) rows."""
     lens = SOFTMAX_LENS
@@ -369,7 +369,7 @@ def _ramp_case():
     pc = synth.make_paged_cache(wl, lens, spare_pages=2)
     for b, Lb in enumerate(lens):
         rows = pc.rows_f32(b, Lb).copy()
-        rows[:, 512:] *= (1.0 + 15.0 * np.arange(Lb) / max(Lb - 1, 1))[:, None]
+        rows[:, 512:] *= (1.0 + 31.0 * np.arange(Lb) / max(Lb - 1, 1))[:, None]
         _set_rows(pc, b, rows)
     return wl, pc, synth.make_q_lat(wl)
 
