@@ -13,10 +13,10 @@
 // weights are streamed once through a TMA ring (weights do not depend on the
 // previous kernel, so the first stages are requested before waiting for it).
 //
-// Per chunk of 64 K columns the ring holds a W_UQ,i tile (128 rows), a W_QR
-// tile (rows 64 i .. 64 i + 127: head i's 64 rows are the first half; the
-// second half belongs to head i + 1 and is discarded, which keeps the MMA at
-// M = 128) and the chunk of x.  After the K loop the same ring carries W_UK,i
+// Per chunk of 64 K columns the ring holds a W_UQ,i tile (128 rows), head i's
+// 64 W_QR rows in the first half of a 128-row tile (the MMA runs at M = 128;
+// the second half holds whatever an earlier chunk left there, and its 64
+// output rows are never read) and the chunk of x.  After the K loop the same ring carries W_UK,i
 // (read MN-major as W_UK,i^T, four 128-row M tiles).  D accumulates in TMEM
 // with a column stride w (the padded batch rounded up to 32): q_C at columns
 // [0, w), q_R at [w, 2w); then q~ tile t at [t w, (t + 1) w), written once the
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const uint32_t tx1 = 2 * kTile + g.n_pad * 128;
+      const uint32_t tx1 = kTile + kTile / 2 + g.n_pad * 128;
       auto load_w = [&](int c, int st) {
         uint8_t *dst = smem + st * g.stage_bytes;
         if (c < nk1) {
@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (quad < 2) {
-      // q_R of this head (TMEM lanes 0..63), unrotated, fp32
+      // q_R of this head (TMEM lanes 0..63), unrotated, fp32; lanes 64..127
+      // come from the unloaded half of the W_QR tile and are not read
       for (int c0 = 0; c0 < g.n_pad; c0 += 32) {
         float v[32];
         tmem_ld32f(tmem + lane_off + g.n_cols + c0, v);
@@ -254,9 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j)
           if (c0 + j < g.n_pad) qr[(c0 + j) * 64 + row] = v[j];
       }
-    } else {
-      // the upper half of the W_QR tile belongs to the next head: read, not used
-      // (every warp runs the same TMEM loads, so the collective form stays aligned)
     }
     fence_proxy_async_smem();              // q_C -> the W_UK MMAs
     tc_fence_before();
@@ -357,7 +355,7 @@ cudaError_t absorb_heads(const __nv_bfloat16 *x, int K, const __nv_bfloat16 *W_U
   if (e != cudaSuccess) return e;
   CUtensorMap tm_uq, tm_qr, tm_uk;
   if (!map2d(&tm_uq, W_UQ, (long)kH * 128, K, 64, 128) ||
-      !map2d(&tm_qr, W_QR, (long)kH * 64, K, 64, 128) ||
+      !map2d(&tm_qr, W_QR, (long)kH * 64, K, 64, 64) ||
       !map2d(&tm_uk, W_UK, (long)kH * 128, 512, 64, 64))
     return cudaErrorInvalidValue;
   // batch rows in chunks of at most 128 (four q~ tiles of n columns fill TMEM)

@@ -78,9 +78,11 @@ cudaError_t absorb_proj(const bf16 *x, const bf16 *W_DQ, const bf16 *W_UQ, const
 
 cudaError_t unabsorb_proj(const bf16 *z, const bf16 *W_UV, const bf16 *W_O, int batch,
                           int d_model, bf16 *o, bf16 *out, int *err, cudaStream_t s) {
-  // o_i = W_UV,i z_i: per head, K = 512
+  // o_i = W_UV,i z_i: per head, K = 512 (split in-cluster: one 128-row tile per
+  // head leaves each CTA a short serial chain otherwise)
   GemmOp u = op(W_UV, 128, kH, 0);
   direct(u, kOutBf16, W_O ? o : out, (long)kH * 128, 128);
+  cluster_split(u, gemm_cluster_splits(1, kH, 512 / 64));
   TRY(gemm(&u, 1, z, batch, (long)kH * 512, 512, 512, err, s));
   if (!W_O) return cudaSuccess;
   // u = W_O o, its K splits summed in-cluster

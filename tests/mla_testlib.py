@@ -18,6 +18,11 @@ from mla_latent_kv_45_b200 import synth
 BF16_MAX_ABS = 2e-2
 BF16_MEAN_REL = 5e-3
 FP32_REL = 1e-4
+# lse of the bf16 path: the kernels sum the bf16-rounded P values the MMA
+# consumes, each within 2^-9 relative of the exact weight, so l may be off by a
+# factor (1 + d), |d| <= 2^-9, and lse by ln(1 + 2^-9) = 1.95e-3, plus fp32
+# score rounding and the approximate exp2 / log2 (~1e-4 at these logit sizes).
+LSE_ATOL = 3e-3
 
 
 def lib_dims(wl: synth.Workload, **kw) -> L.Dims:
