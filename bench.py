@@ -16,10 +16,12 @@ the workload's shape; weights N(0, 0.02^2).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
-The timed region replays the step captured once as a CUDA graph (the same
-launches the eager calls make); a second, eager pass records per-call CUDA
-events for the breakdown and the attention call's roofline, and a third pass
-measures the end-to-end number through the Python API with host buffers.
+The timed region replays the step captured once as a CUDA graph through the
+Python API (``DecodeLayer.capture`` -> ``StepGraph.replay``: the same launches
+the eager calls make); a second, eager pass records per-call CUDA events for
+the breakdown and the attention call's roofline, and a third pass measures the
+end-to-end number: pinned host copies of each step's inputs, the replay and
+the copy of the output back, all on the device clock.
 
 Multi-GPU: ``--gpus N`` starts N ranks on this node (one per GPU, NCCL),
 data-parallel over sequences, each rank its own batch (weak scaling), no
@@ -295,7 +297,7 @@ def run_mine(args):
     import torch
     from mla_latent_kv_45_b200 import _lib as L
     from mla_latent_kv_45_b200 import build, synth
-    from mla_latent_kv_45_b200.layer import DecodeLayer
+    from mla_latent_kv_45_b200.layer import DecodeLayer, StepGraph
 
     rank, world, local = setup_dist(args)
     torch.cuda.set_device(local)
@@ -330,15 +332,21 @@ def run_mine(args):
         z = torch.empty(wl.batch, wl.n_heads, wl.d_c, dtype=torch.bfloat16, device=dev)
         lse = torch.empty(wl.batch, wl.n_heads, dtype=torch.float32, device=dev)
 
-        def step(e=None):
+        def step(e=None, st=None):
+            st = st or stream
             if e:
-                e[4].record(stream)
-            L.mla_decode_attn(dims, cache, q_dev, z, lse, args.num_splits, ws, stream)
+                e[4].record(st)
+            L.mla_decode_attn(dims, cache, q_dev, z, lse, args.num_splits, ws, st)
             if e:
-                e[5].record(stream)
+                e[5].record(st)
 
         def device_error():
             return L.mla_get_device_error(ws)
+
+        def capture():
+            step()
+            torch.cuda.synchronize()
+            return StepGraph(lambda st: step(st=st), z)
 
         inputs, output = [q_dev], z
         launches = LAUNCHES_ATTENTION
@@ -351,6 +359,9 @@ def run_mine(args):
         def step(e=None):
             layer.step(cache, hd, pos, stream, e)
 
+        def capture():
+            return layer.capture(cache, hd, pos)
+
         device_error = layer.device_error
         inputs, output = [hd, pos, cache.seq_lens], layer.out
         launches = LAUNCHES_FULL_STEP
@@ -362,17 +373,9 @@ def run_mine(args):
     if st != 0:
         raise RuntimeError(f"device error {L.STATUS.get(st)} during warm-up")
 
-    # one step captured as a CUDA graph (the same launches, replayed)
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream(device=dev)
-    cap.wait_stream(stream)
-    with torch.cuda.stream(cap):
-        stream_saved = stream
-        stream = cap
-        with torch.cuda.graph(graph, stream=cap):
-            step()
-        stream = stream_saved
-    stream.wait_stream(cap)
+    # one step captured as a CUDA graph through the Python API (the same
+    # launches, replayed with no per-kernel host work)
+    graph = capture()
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()
@@ -418,14 +421,15 @@ def run_mine(args):
                               e[4].elapsed_time(e[5]), e[5].elapsed_time(e[6])] for e in ev])
 
     # ---- end-to-end through the Python API with host buffers: pinned h2d of the
-    # step's inputs and d2h of its output inside the timed region, eager calls
+    # step's inputs into the captured step's buffers, the replay, and the d2h of
+    # its output, all inside the timed region
     host_in = [t.cpu().pin_memory() for t in inputs]
     out_host = torch.empty(output.shape, dtype=output.dtype).pin_memory()
 
     def e2e_step():
         for d, hbuf in zip(inputs, host_in):
             d.copy_(hbuf, non_blocking=True)
-        step()
+        graph.replay()
         out_host.copy_(output, non_blocking=True)
 
     for _ in range(3):
@@ -475,7 +479,7 @@ def run_mine(args):
                    "global_batch": wl.batch * world, "cached_rows_per_step": alg["rows"],
                    "parallelism": f"dp{world} (sequences sharded, no collective)",
                    "l2": l2, "num_splits": args.num_splits,
-                   "timed": "one captured CUDA graph of the step, replayed K times"},
+                   "timed": "the step captured once (DecodeLayer.capture), replayed K times"},
         "roofline": {"kernel": "mla_decode_attn (plan + attention + split merge)",
                      "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak,
@@ -491,7 +495,8 @@ def run_mine(args):
         "e2e": {"value": alg["rows"] * wl.n_heads * world / (e2e_ms / args.steps / 1e3),
                 "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms / args.steps,
-                "how": "eager API calls per step, pinned host copies in and out on the stream"},
+                "how": "per step: pinned host copies of the inputs into the step's buffers, "
+                       "StepGraph.replay(), pinned copy of the output back, one stream"},
         "gpu_launches": launches * args.steps,
     }
     if rank == 0:

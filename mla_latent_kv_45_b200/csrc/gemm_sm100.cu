@@ -16,8 +16,10 @@
 //  * X (the activations, bf16) is reloaded from L2 per K chunk;
 //  * two problems that share X (e.g. W_DKV and W_KR, W_UQ and W_QR) run in one
 //    launch; per-head problems (W_UK, W_UV) index heads in their items;
-//  * the epilogue writes bf16 / fp32 outputs directly or fp32 split-K
-//    partials that are summed in a fixed order (deterministic).
+//  * the epilogue writes bf16 / fp32 outputs directly; where there are too few
+//    tiles, the K range of each tile is split across the CTAs of a cluster,
+//    which sum their partial tiles through distributed shared memory in a
+//    fixed order (deterministic).
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocation + MMA issue,
 // warps 2-5 epilogue.  Every wait is bounded (globaltimer).
 #include <cuda.h>
@@ -242,16 +244,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int n = c + j;
             if (n < g.n) {
               const float v = __uint_as_float(r[j]);
-              if (P.out_mode == kOutPartial) {
-                P.part[((long)it.split * g.n_total + g.n0 + n) * P.part_ld + P.part_col +
-                       (long)it.head * P.M + m] = v;
-              } else {
-                const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
-                if (P.out_mode == kOutBf16)
-                  static_cast<__nv_bfloat16 *>(P.out)[idx] = __float2bfloat16_rn(v);
-                else
-                  static_cast<float *>(P.out)[idx] = v;
-              }
+              const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
+              if (P.out_mode == kOutBf16)
+                static_cast<__nv_bfloat16 *>(P.out)[idx] = __float2bfloat16_rn(v);
+              else
+                static_cast<float *>(P.out)[idx] = v;
             }
           }
         }
@@ -302,23 +299,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, g.tmem_cols);
-  }
-}
-
-// Y[n][col_off + m] = sum over splits of part[s][n][m]  (bf16 or fp32 output)
-__global__ void gemm_reduce_kernel(const float *part, int splits, int n_rows, int width,
-                                   int part_ld, void *out, long ldy, int out_bf16) {
-  grid_dep_wait();
-  const long total = (long)n_rows * width;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total;
-       i += (long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / width), m = (int)(i % width);
-    float v = 0.f;
-    for (int s = 0; s < splits; ++s) v += part[((long)s * n_rows + n) * part_ld + m];
-    if (out_bf16)
-      static_cast<__nv_bfloat16 *>(out)[(long)n * ldy + m] = __float2bfloat16_rn(v);
-    else
-      static_cast<float *>(out)[(long)n * ldy + m] = v;
   }
 }
 
@@ -446,16 +426,12 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
                  int x_cols_per_head, int *err, cudaStream_t s) {
   if (nops < 1 || nops > 2 || n < 1 || K % 64) return cudaErrorInvalidValue;
   // in-cluster split-K reduction: every op reduces in clusters of the same size
-  const bool cluster = ops[0].cluster_reduce && !ops[0].part && ops[0].splits > 1;
+  const bool cluster = ops[0].splits > 1;
   for (int i = 0; i < nops; ++i) {
     const GemmOp &o = ops[i];
-    if (!cluster) {
-      if (o.cluster_reduce && !o.part && o.splits > 1) return cudaErrorInvalidValue;
-      continue;
-    }
-    if (!o.cluster_reduce || o.part || o.splits != ops[0].splits ||
-        o.splits > kMaxClusterSplits || (o.M % 4) || (o.ldy % 4) || (o.y_head % 4) ||
-        o.out_mode == kOutPartial || (reinterpret_cast<uintptr_t>(o.out) & 15))
+    if (o.splits != ops[0].splits || o.splits < 1) return cudaErrorInvalidValue;
+    if (cluster && (o.splits > kMaxClusterSplits || (o.M % 4) || (o.ldy % 4) ||
+                    (o.y_head % 4) || (reinterpret_cast<uintptr_t>(o.out) & 15)))
       return cudaErrorInvalidValue;
   }
   const int n_step = cluster ? 128 : 256;
@@ -489,21 +465,14 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
       P.a_mn = o.a_mn;
       P.a_map = i;
       P.a_rows_per_head = o.a_mn ? K : o.M;
-      P.splits = (o.part || cluster) ? o.splits : 1;
+      P.splits = o.splits;
       P.chunks_per_split = (g.k_chunks + P.splits - 1) / P.splits;
       P.item_begin = items;
       items += P.m_tiles * P.splits * o.heads;
-      P.out_mode = o.part ? kOutPartial : o.out_mode;
-      P.out = o.out;
+      P.out_mode = o.out_mode;
       P.ldy = o.ldy;
       P.y_head = o.y_head;
-      P.part = o.part;
-      P.part_ld = o.part_ld;
-      P.part_col = o.part_col;
-      if (P.out_mode != kOutPartial) {
-        const long esz = P.out_mode == kOutBf16 ? 2 : 4;
-        P.out = static_cast<char *>(o.out) + (long)n0 * o.ldy * esz;
-      }
+      P.out = static_cast<char *>(o.out) + (long)n0 * o.ldy * (P.out_mode == kOutBf16 ? 2 : 4);
       const long a_rows = o.a_mn ? (long)o.heads * K : (long)o.heads * o.M;
       const long a_cols = o.a_mn ? o.M : K;
       if (!map2d(&tm[i], o.A, a_rows, a_cols, 64, o.a_mn ? 64 : 128)) return cudaErrorInvalidValue;
@@ -531,15 +500,6 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
-}
-
-cudaError_t gemm_reduce(const float *part, int splits, int n, int width, int part_ld, void *out,
-                        long ldy, bool out_bf16, cudaStream_t s) {
-  const long total = (long)n * width;
-  int blocks = (int)((total + 255) / 256);
-  if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
-  return launch_pdl(gemm_reduce_kernel, dim3(blocks), dim3(256), 0, s, part, splits, n, width,
-                    part_ld, out, ldy, (int)(out_bf16 ? 1 : 0));
 }
 
 }  // namespace sm100

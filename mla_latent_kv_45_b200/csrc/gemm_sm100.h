@@ -8,29 +8,24 @@ namespace mla {
 namespace sm100 {
 
 constexpr int kMaxGemmStages = 8;
-enum : int { kOutPartial = 0, kOutBf16 = 1, kOutF32 = 2 };
+enum : int { kOutBf16 = 1, kOutF32 = 2 };
 
 // One projection Y[n][m] = sum_k A[m][k] X[n][k] (per head when heads > 1).
 //   a_mn = 0: A[m][k] = A2d[head * M + m][k]     (A2d is [heads*M][K], an [out][in] weight)
 //   a_mn = 1: A[m][k] = A2d[head * K + k][m]     (A2d is [heads*K][M], a transposed view)
-// Output (out_mode kOutBf16 / kOutF32): out[n * ldy + head * y_head + m].
-// With part != nullptr the K range is cut into `splits` pieces and each writes
-// fp32 partials part[(split * n_total + n) * part_ld + part_col + head * M + m];
-// gemm_reduce sums them.
-// With cluster_reduce (part == nullptr, 2 <= splits <= kMaxClusterSplits, M,
-// ldy and y_head multiples of 4) the `splits` CTAs of one tile form a thread-
-// block cluster and sum their partial tiles through distributed shared memory
-// in a fixed order, writing the direct output; no partial buffer, no reduce
-// launch.  Every op of a launch must then use the same splits.
+// Output: out[n * ldy + head * y_head + m], bf16 or fp32.
+// With splits > 1 (at most kMaxClusterSplits; M, ldy and y_head multiples of
+// 4, out 16-byte aligned) the K range of each tile is cut into `splits` CTAs
+// that form a thread-block cluster and sum their partial tiles through
+// distributed shared memory in a fixed order.  Every op of a launch uses the
+// same splits.
 struct GemmOp {
   const __nv_bfloat16 *A;
   int M, heads, a_mn;
   int out_mode;
   void *out;
   long ldy, y_head;
-  float *part;
-  int part_ld, part_col, splits;
-  int cluster_reduce;
+  int splits;
 };
 
 constexpr int kMaxClusterSplits = 8;
@@ -41,8 +36,6 @@ struct GemmProblem {
   int M, m_tiles, a_mn, a_map, a_rows_per_head, splits, chunks_per_split, item_begin, out_mode;
   void *out;
   long ldy, y_head;
-  float *part;
-  int part_ld, part_col;
 };
 
 struct GemmLaunch {
@@ -63,10 +56,6 @@ int gemm_splits(int m_tiles, int heads, int k_chunks);
 // columns [h * x_cols_per_head, ... + K)).  K must be a multiple of 64.
 cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, long x_cols, int K,
                  int x_cols_per_head, int *err, cudaStream_t s);
-
-// out[n * ldy + m] = sum_s part[(s * n_rows + n) * part_ld + m], m < width.
-cudaError_t gemm_reduce(const float *part, int splits, int n_rows, int width, int part_ld,
-                        void *out, long ldy, bool out_bf16, cudaStream_t s);
 
 }  // namespace sm100
 }  // namespace mla

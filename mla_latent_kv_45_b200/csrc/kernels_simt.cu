@@ -309,9 +309,7 @@ cudaError_t launch_rope_q(const float *qr, int batch, int n_heads, int d_c, cons
 }
 template cudaError_t launch_rope_q<float>(const float *, int, int, int, const RopeParams &,
                                           const int32_t *, float *, cudaStream_t);
-template cudaError_t launch_rope_q<__nv_bfloat16>(const float *, int, int, int,
-                                                  const RopeParams &, const int32_t *,
-                                                  __nv_bfloat16 *, cudaStream_t);
+
 
 // ---------------------------------------------------------------------------
 // Plan: balanced split of the batch's pages into partitions

@@ -35,14 +35,10 @@ void direct(GemmOp &o, int mode, void *out, long ldy, long y_head = 0) {
   o.out = out;
   o.ldy = ldy;
   o.y_head = y_head;
-  o.part = nullptr;
 }
 
 // the K range cut into `splits` CTAs that sum their partial tiles in-cluster
-void cluster_split(GemmOp &o, int splits) {
-  o.splits = splits;
-  o.cluster_reduce = splits > 1;
-}
+void cluster_split(GemmOp &o, int splits) { o.splits = splits; }
 
 }  // namespace
 

@@ -79,8 +79,43 @@ class DecodeLayer:
             events[6].record(main)
         return self.out
 
+    def capture(self, cache: L.PagedCache, h: torch.Tensor, positions: torch.Tensor
+                ) -> "StepGraph":
+        """The decode step over these buffers, captured once as a CUDA graph.
+
+        The graph reads ``h``, ``positions``, ``cache.seq_lens`` and the cache
+        in place and writes ``self.out`` (and the cache row): copy each step's
+        inputs into those buffers and call ``replay()``.  One eager step runs
+        first so that every one-time set-up (per-device kernel attributes)
+        happens outside the capture.
+        """
+        self.step(cache, h, positions)
+        torch.cuda.synchronize()
+        return StepGraph(lambda s: self.step(cache, h, positions, s), self.out)
+
     def device_error(self) -> int:
         """Synchronises; returns the first nonzero device status of both workspaces."""
         st = L.mla_get_device_error(self.ws_append, self.side)
         st2 = L.mla_get_device_error(self.ws)
         return st if st != 0 else st2
+
+
+class StepGraph:
+    """A CUDA graph of one call sequence issued by ``fn(stream)``; ``replay``
+    launches the same kernels on the current stream with no per-kernel host
+    work."""
+
+    def __init__(self, fn, out: torch.Tensor):
+        self.out = out
+        self.graph = torch.cuda.CUDAGraph()
+        main = torch.cuda.current_stream()
+        cap = torch.cuda.Stream(device=main.device)
+        cap.wait_stream(main)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(self.graph, stream=cap):
+                fn(cap)
+        main.wait_stream(cap)
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.out

@@ -20,9 +20,13 @@ BF16_MEAN_REL = 5e-3
 FP32_REL = 1e-4
 # lse of the bf16 path: the kernels sum the bf16-rounded P values the MMA
 # consumes, each within 2^-9 relative of the exact weight, so l may be off by a
-# factor (1 + d), |d| <= 2^-9, and lse by ln(1 + 2^-9) = 1.95e-3, plus fp32
-# score rounding and the approximate exp2 / log2 (~1e-4 at these logit sizes).
+# factor (1 + d), |d| <= 2^-9, and lse by ln(1 + 2^-9) = 1.95e-3, plus the
+# approximate exp2 / log2 (~1e-6).  On top of that the raw scores are fp32 sums
+# of 576 products accumulated by the tensor core in its own order; that error
+# scales with the logits' size, hence a relative term (logits of ~50 nats in
+# the rescale test showed 3.5e-3 in all).
 LSE_ATOL = 3e-3
+LSE_RTOL = 5e-5
 
 
 def lib_dims(wl: synth.Workload, **kw) -> L.Dims:
