@@ -85,10 +85,20 @@ def attention_only(wl) -> bool:
     return wl.new_tokens == 0
 
 
+def prefill(wl) -> bool:
+    """A chunk of new tokens per sequence: run as one entry per token sharing the
+    sequence's page-table row, entry t attending to rows 0 .. p0 + t."""
+    return wl.new_tokens > 1
+
+
 def describe(wl):
     if attention_only(wl):
         what = "latent attention only (plan + attention + split merge) over the cached rows"
         rows = f"{wl.prior_min} rows per sequence (the query's own included)"
+    elif prefill(wl):
+        what = ("chunked prefill through the decode calls: the chunk's tokens as entries "
+                "sharing the page table row (causal), append + absorb_q + attention + unabsorb")
+        rows = f"{wl.prior_min} cached rows + a {wl.new_tokens}-token chunk"
     else:
         what = "full layer step: append + absorb_q (W_DQ) + attention + unabsorb (W_UV, W_O)"
         rows = f"cached rows {wl.prior_min}..{wl.prior_max} + {wl.new_tokens} new"
@@ -105,15 +115,24 @@ def row_bytes(wl):
 
 
 def attended_lengths(wl, prior):
-    """Rows each sequence's query attends to."""
-    return prior if attention_only(wl) else prior + 1
+    """Rows each query attends to (per token of a prefill chunk)."""
+    if attention_only(wl):
+        return prior
+    if prefill(wl):
+        return np.concatenate([p + 1 + np.arange(wl.new_tokens) for p in prior])
+    return prior + 1
 
 
 def algorithmic(wl, lens):
     """Bytes / FLOPs that any implementation must move / do, per step and per attention call."""
-    B, H = wl.batch, wl.n_heads
+    B, H = len(lens), wl.n_heads      # queries (a prefill chunk's tokens count one each)
     rows = int(lens.sum())
-    attn_bytes = rows * row_bytes(wl) + B * H * 576 * 2 + B * H * 512 * 2   # cache + q_lat + z
+    if prefill(wl):
+        # each cached row is needed once per chunk, not once per query
+        cached = int(wl.batch * (wl.prior_max + wl.new_tokens))
+        attn_bytes = cached * row_bytes(wl) + B * H * 576 * 2 + B * H * 512 * 2
+    else:
+        attn_bytes = rows * row_bytes(wl) + B * H * 576 * 2 + B * H * 512 * 2  # cache + q_lat + z
     attn_flops = rows * H * FLOP_PER_ROW_HEAD
     if attention_only(wl):
         return dict(rows=rows, attn_bytes=attn_bytes, attn_flops=attn_flops,
@@ -352,9 +371,18 @@ def run_mine(args):
         launches = LAUNCHES_ATTENTION
     else:
         Wd = {k: (None if v is None else bf(v)) for k, v in W.items()}
-        hd = bf(h)
-        pos = torch.from_numpy(prior.astype(np.int32)).to(dev)
-        layer = DecodeLayer(dims, Wd, wl.batch, args.num_splits, device=dev)
+        if prefill(wl):
+            # one entry per chunk token, all sharing their sequence's page-table row
+            T = wl.new_tokens
+            hd = bf(synth.make_hidden(wl, n=wl.batch * T))
+            pos = torch.from_numpy(np.concatenate([p + np.arange(T) for p in prior])
+                                   .astype(np.int32)).to(dev)
+            cache = L.PagedCache(pool, torch.from_numpy(np.repeat(pc.block_table, T, axis=0))
+                                 .to(dev), torch.from_numpy(lens.astype(np.int32)).to(dev))
+        else:
+            hd = bf(h)
+            pos = torch.from_numpy(prior.astype(np.int32)).to(dev)
+        layer = DecodeLayer(dims, Wd, len(lens), args.num_splits, device=dev)
 
         def step(e=None):
             layer.step(cache, hd, pos, stream, e)

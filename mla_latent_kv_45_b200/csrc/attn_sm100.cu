@@ -398,33 +398,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float pend_sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     // chunk idx (in `slot`) landed: int8 codes of page sp at +8 KB + 4 KB sp, row r
     // at 64 r; bf16 out at +8 KB sp, row r at 128 r, 16-byte unit u at (u ^ (r & 7)) << 4.
-    // Eight passes per page, pass i converting rows 8i..8i+7 with lane l on input
-    // unit 32 i + l (consecutive 16-byte reads, no bank conflict; the two output
-    // units of the 4 lanes of a row are even and odd, rows alternate, so the
-    // stores do not conflict either).  Page 1's output covers page 0's input
-    // and, from row 32 on, its own rows 16 i - 64 .. 16 i - 49, all read in
-    // earlier passes or before this pass's writes: page 0 is converted first
-    // and every pass is read before it is written.
+    // Page 1's output covers page 0's input and, from row 32 on, its own: page 0
+    // is converted first, and every 32-row batch is read before it is written.
     auto finish_k = [&](int slot, int idx, int c, const bool (&has)[2],
                         const float (&sc)[2][2]) -> bool {
       if (!wait_bar(ctx, &bars->k_land[slot], (idx / kKSlots) & 1)) return false;
       if (c < 8) {
         uint8_t *base = smem + kOffK + slot * kKChunk;
-        const int jj = lane & 3;
         for (int sp = 0; sp < 2; ++sp) {
           if (!has[sp]) continue;
-          // this lane's rows 8 i + lane / 4: their scales, from the lanes that hold them
-          for (int i = 0; i < 8; ++i) {
-            const int r = 8 * i + (lane >> 2);
-            const float scale = __shfl_sync(0xffffffffu, sc[sp][r >> 5], r & 31);
-            const uint4 v =
-                reinterpret_cast<const uint4 *>(base + 8192 + 4096 * sp)[32 * i + lane];
+          for (int hf = 0; hf < 2; ++hf) {
+            const int r = 32 * hf + lane;
+            const uint4 *in = reinterpret_cast<const uint4 *>(base + 8192 + 4096 * sp + 64 * r);
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[j] = in[j];
             __syncwarp();
-            uint4 lo, hi;
-            i8x16_to_bf16(v, scale, lo, hi);
             uint8_t *out = base + kBox * sp + 128 * r;
-            *reinterpret_cast<uint4 *>(out + (((2 * jj) ^ (r & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4 *>(out + (((2 * jj + 1) ^ (r & 7)) << 4)) = hi;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 lo, hi;
+              i8x16_to_bf16(v[j], sc[sp][hf], lo, hi);
+              *reinterpret_cast<uint4 *>(out + (((2 * j) ^ (r & 7)) << 4)) = lo;
+              *reinterpret_cast<uint4 *>(out + (((2 * j + 1) ^ (r & 7)) << 4)) = hi;
+            }
             __syncwarp();
           }
         }
@@ -577,30 +574,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!wait_bar(ctx, &bars->v_land[slot], (idx / kVSlots) & 1)) return false;
       if (kI8) {
         // int8 codes of row r at +8 KB + 128 r (128 latent columns) -> bf16 boxes
-        // 0 (columns 0-63) at 128 r and 1 (64-127) at 8 KB + 128 r.  Pass i
-        // converts rows 4i..4i+3, lane l on input unit 32 i + l (row 4 i + l / 8,
-        // columns 16 (l % 8) ..): consecutive reads; box 1's row r is exactly the
-        // input row r, read by the pass before the pass writes.  The lanes of a row
-        // with l % 8 >= 4 (box 1) store their odd unit first, so the two boxes'
-        // stores of a pass fall in different banks.
+        // 0 (columns 0-63) at 128 r and 1 (64-127) at 8 KB + 128 r: box 1's row r is
+        // exactly the input row r, which the lane has read before it writes
         uint8_t *dst = smem + kOffV + slot * kVChunk;
-        const int j = lane & 7, bx = j >> 2, u = 2 * (j & 3);
-        for (int i = 0; i < 16; ++i) {
-          const int r = 4 * i + (lane >> 3);
-          const float scale = __shfl_sync(0xffffffffu, r < 32 ? sc0 : sc1, r & 31);
-          const uint4 v = reinterpret_cast<const uint4 *>(dst + kBox)[32 * i + lane];
-          __syncwarp();
-          uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
-          if (r < valid) i8x16_to_bf16(v, scale, lo, hi);
-          uint8_t *out = dst + bx * kBox + 128 * r;
-          if (bx) {
-            *reinterpret_cast<uint4 *>(out + (((u + 1) ^ (r & 7)) << 4)) = hi;
-            *reinterpret_cast<uint4 *>(out + ((u ^ (r & 7)) << 4)) = lo;
-          } else {
+        for (int hf = 0; hf < 2; ++hf) {
+          const int r = 32 * hf + lane;
+          const float sc = hf ? sc1 : sc0;
+          uint4 v[8];
+          const uint4 *in = reinterpret_cast<const uint4 *>(dst + kBox + 128 * r);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = in[j];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+            if (r < valid) i8x16_to_bf16(v[j], sc, lo, hi);
+            uint8_t *out = dst + (j >> 2) * kBox + 128 * r;
+            const int u = 2 * (j & 3);
             *reinterpret_cast<uint4 *>(out + ((u ^ (r & 7)) << 4)) = lo;
             *reinterpret_cast<uint4 *>(out + (((u + 1) ^ (r & 7)) << 4)) = hi;
           }
-          __syncwarp();
         }
         fence_proxy_async_smem();
       } else if (valid < kPage) {

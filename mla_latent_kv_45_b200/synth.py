@@ -18,6 +18,7 @@ Workloads (DeepSeek-V2 attention sizes from "从零理解 MLA", 实际配置:
              the query's own row included), attention only.
 * ``v2_step128`` bf16, batch 128, 2048 cached rows + 1 new, whole layer step.
 * ``v2_batch64_int8``  ``v2_batch64`` over 656-byte int8 cache rows.
+* ``v2_prefill256``    one sequence, 4096 cached rows, a 256-token chunk.
 
 Distributions: weights N(0, 0.02^2), hidden states N(0, 1), RMSNorm gain 1
 (optionally 1 + 0.1 N(0,1)), cached rows N(0, 1) (the scale of an
@@ -77,7 +78,7 @@ class Workload:
     dtype: str               # "bf16" | "fp32"
     prior_min: int           # cached rows before the step, per sequence
     prior_max: int
-    new_tokens: int = 1      # 1 = one appended token; 0 = attention only
+    new_tokens: int = 1      # new tokens per sequence (a chunk when > 1); 0 = attention only
     shuffle_pages: bool = True
     rope_base: float = 10000.0
     rms_eps: float = 1e-6
@@ -97,9 +98,12 @@ V2_LONG = Workload("v2_long", 3, 8, 128, 5120, 1536, 512, 128, 64, 128, 64, "bf1
 V2_STEP128 = Workload("v2_step128", 4, 128, 128, 5120, 1536, 512, 128, 64, 128, 64, "bf16", 2048, 2048)
 # the batch-64 workload (same seeds) over an int8 latent cache
 V2_BATCH64_INT8 = dataclasses.replace(V2_BATCH64, name="v2_batch64_int8", cache="int8")
+# chunked prefill: one sequence, 4096 cached rows, a chunk of 256 new tokens
+V2_PREFILL256 = Workload("v2_prefill256", 6, 1, 128, 5120, 1536, 512, 128, 64, 128, 64, "bf16",
+                         4096, 4096, new_tokens=256)
 
 WORKLOADS = {w.name: w for w in (TINY, V2_SINGLE, V2_BATCH64, V2_LONG, V2_STEP128,
-                                 V2_BATCH64_INT8)}
+                                 V2_BATCH64_INT8, V2_PREFILL256)}
 
 
 def reduced(base: Workload, name: str, wid: int, batch: int, prior_min: int, prior_max: int,
