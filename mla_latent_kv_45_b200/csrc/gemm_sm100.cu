@@ -369,31 +369,44 @@ cudaError_t set_smem_attr() {
   });
 }
 
-// Clusters of `size` CTAs (two CTAs' worth of shared memory per SM) that the
-// device can hold at once, or 0 if that cannot be determined (queried once per
-// device and size).
-int max_active_clusters(int size) {
+// Pipeline stages and dynamic shared memory of a launch with n_pad batch
+// columns: two CTAs per SM, each with at most half of the 227 KB.
+int stages_for(int n_pad) {
+  const int stage_bytes = kABytes + n_pad * 128;
+  int st = (232448 / 2 - 1024 - 256) / stage_bytes;
+  return st > kMaxGemmStages ? kMaxGemmStages : st;
+}
+size_t smem_for(int n_pad) {
+  return (size_t)stages_for(n_pad) * (kABytes + n_pad * 128) + 256 + 1024;
+}
+
+// Clusters of `size` CTAs of a launch with n_pad batch columns that the device
+// can hold at once, or 0 if that cannot be determined (queried once per device,
+// size and padded batch).
+int max_active_clusters(int size, int n_pad) {
   static std::mutex lock;
-  static int known[64][kMaxClusterSplits + 1];
+  static int known[64][kMaxClusterSplits + 1][9];
   static bool init = false;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || size < 1 ||
-      size > kMaxClusterSplits)
+      size > kMaxClusterSplits || n_pad < 16 || n_pad > 128 || n_pad % 16)
     return 0;
+  const int ni = n_pad / 16;
   {
     std::lock_guard<std::mutex> g(lock);
     if (!init) {
-      for (auto &row : known)
-        for (int &v : row) v = -1;
+      for (auto &a : known)
+        for (auto &b : a)
+          for (int &v : b) v = -1;
       init = true;
     }
-    if (known[dev][size] >= 0) return known[dev][size];
+    if (known[dev][size][ni] >= 0) return known[dev][size][ni];
   }
   if (set_smem_attr() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(size);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 232448 / 2 - 256;
+  cfg.dynamicSmemBytes = smem_for(n_pad);
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = size;
@@ -404,20 +417,23 @@ int max_active_clusters(int size) {
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, gemm_sm100_kernel, &cfg) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> g(lock);
-  known[dev][size] = n;
+  known[dev][size][ni] = n;
   return n;
 }
 
 }  // namespace
 
-int gemm_cluster_splits(int m_tiles, int heads, int k_chunks) {
+int gemm_cluster_splits(int m_tiles, int heads, int k_chunks, int n) {
   int s = gemm_splits(m_tiles, heads, k_chunks);
   if (s > kMaxClusterSplits) s = kMaxClusterSplits;
   // one cluster per tile: take the largest split whose clusters all fit on the
-  // device at once (clusters live inside one GPC, so a size that packs badly
-  // would leave some tiles for a second wave)
+  // device at once, for the shared memory these launches use (clusters live
+  // inside one GPC, so a size that packs badly would leave some tiles for a
+  // second wave)
   const int tiles = m_tiles * heads;
-  while (s > 2 && max_active_clusters(s) < tiles) --s;
+  const int nn = n < 128 ? n : 128;   // cluster launches take the batch in chunks of 128
+  const int n_pad = (nn + 15) / 16 * 16;
+  while (s > 2 && max_active_clusters(s, n_pad) < tiles) --s;
   const int per = (k_chunks + s - 1) / s;
   return (k_chunks + per - 1) / per;
 }
@@ -452,8 +468,7 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     while (g.tmem_cols < 2 * g.n_cols) g.tmem_cols *= 2;
     const int stage_bytes = kABytes + g.n_pad * 128;
     // two CTAs per SM: half of the 227 KB of shared memory each
-    g.stages = (232448 / 2 - 1024 - 256) / stage_bytes;
-    if (g.stages > kMaxGemmStages) g.stages = kMaxGemmStages;
+    g.stages = stages_for(g.n_pad);
     CUtensorMap tm[2], tx;
     int items = 0;
     g.nprob = nops;
@@ -480,7 +495,7 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     if (nops == 1) tm[1] = tm[0];
     if (!map2d(&tx, X + (long)n0 * x_cols, nn, x_cols, 64, g.n_pad)) return cudaErrorInvalidValue;
     g.items = items;
-    const size_t smem = (size_t)g.stages * stage_bytes + 256 + 1024;
+    const size_t smem = smem_for(g.n_pad);
     cudaError_t e;
     if (cluster) {
       // one item per CTA; the splits of a tile form one cluster and their

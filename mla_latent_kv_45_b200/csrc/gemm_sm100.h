@@ -46,8 +46,9 @@ struct GemmLaunch {
   int *err;
 };
 
-// Split count for an in-cluster reduction (at most kMaxClusterSplits).
-int gemm_cluster_splits(int m_tiles, int heads, int k_chunks);
+// Split count for an in-cluster reduction (at most kMaxClusterSplits) of a
+// problem with m_tiles x heads tiles, K / 64 chunks and batch n.
+int gemm_cluster_splits(int m_tiles, int heads, int k_chunks, int n);
 
 // Split count for a problem of m_tiles x heads tiles and K / 64 chunks.
 int gemm_splits(int m_tiles, int heads, int k_chunks);

@@ -45,7 +45,7 @@ void cluster_split(GemmOp &o, int splits) { o.splits = splits; }
 cudaError_t append_proj(const bf16 *h, const bf16 *W_DKV, const bf16 *W_KR, int batch,
                         int d_model, float *xkv, int *err, cudaStream_t s) {
   // [W_DKV h ; W_KR h] in fp32, its K splits summed in-cluster
-  const int splits = gemm_cluster_splits(5, 1, d_model / 64);
+  const int splits = gemm_cluster_splits(5, 1, d_model / 64, batch);
   GemmOp ops[2] = {op(W_DKV, 512, 1, 0), op(W_KR, 64, 1, 0)};
   direct(ops[0], kOutF32, xkv, 576);
   direct(ops[1], kOutF32, xkv + 512, 576);
@@ -63,7 +63,7 @@ cudaError_t absorb_proj(const bf16 *x, const bf16 *W_DQ, const bf16 *W_UQ, const
     // c_Q = W_DQ h, its K splits summed in-cluster
     GemmOp o = op(W_DQ, d_q, 1, 0);
     direct(o, kOutBf16, cq, d_q);
-    cluster_split(o, gemm_cluster_splits((d_q + 127) / 128, 1, d_in / 64));
+    cluster_split(o, gemm_cluster_splits((d_q + 127) / 128, 1, d_in / 64, batch));
     TRY(gemm(&o, 1, x, batch, d_in, d_in, 0, err, s));
     xin = cq;
   }
@@ -78,13 +78,13 @@ cudaError_t unabsorb_proj(const bf16 *z, const bf16 *W_UV, const bf16 *W_O, int 
   // head leaves each CTA a short serial chain otherwise)
   GemmOp u = op(W_UV, 128, kH, 0);
   direct(u, kOutBf16, W_O ? o : out, (long)kH * 128, 128);
-  cluster_split(u, gemm_cluster_splits(1, kH, 512 / 64));
+  cluster_split(u, gemm_cluster_splits(1, kH, 512 / 64, batch));
   TRY(gemm(&u, 1, z, batch, (long)kH * 512, 512, 512, err, s));
   if (!W_O) return cudaSuccess;
   // u = W_O o, its K splits summed in-cluster
   GemmOp w = op(W_O, d_model, 1, 0);
   direct(w, kOutBf16, out, d_model);
-  cluster_split(w, gemm_cluster_splits((d_model + 127) / 128, 1, kH * 128 / 64));
+  cluster_split(w, gemm_cluster_splits((d_model + 127) / 128, 1, kH * 128 / 64, batch));
   return gemm(&w, 1, o, batch, kH * 128, kH * 128, 0, err, s);
 }
 
