@@ -367,6 +367,19 @@ def run_mine(args):
             torch.cuda.synchronize()
             return StepGraph(lambda st: step(st=st), z)
 
+        def second_set():
+            # its own input, output and workspace buffers over the same cache
+            q2, z2, l2 = q_dev.clone(), torch.empty_like(z), torch.empty_like(lse)
+            ws2 = torch.empty_like(ws)
+            L.mla_workspace_init(ws2)
+
+            def run(st):
+                L.mla_decode_attn(dims, cache, q2, z2, l2, args.num_splits, ws2, st)
+
+            run(stream)
+            torch.cuda.synchronize()
+            return StepGraph(run, z2), [q2], z2, lambda: L.mla_get_device_error(ws2)
+
         inputs, output = [q_dev], z
         launches = LAUNCHES_ATTENTION
     else:
@@ -389,6 +402,15 @@ def run_mine(args):
 
         def capture():
             return layer.capture(cache, hd, pos)
+
+        def second_set():
+            # another layer object (workspaces, outputs) over the same weights and
+            # pool, with its own input buffers and sequence lengths
+            layer2 = DecodeLayer(dims, Wd, len(lens), args.num_splits, device=dev)
+            h2, p2 = hd.clone(), pos.clone()
+            cache2 = L.PagedCache(cache.pool, cache.block_table, cache.seq_lens.clone())
+            return (layer2.capture(cache2, h2, p2), [h2, p2, cache2.seq_lens], layer2.out,
+                    layer2.device_error)
 
         device_error = layer.device_error
         inputs, output = [hd, pos, cache.seq_lens], layer.out
@@ -448,35 +470,58 @@ def run_mine(args):
         per_call = np.array([[e[0].elapsed_time(e[1]), e[2].elapsed_time(e[3]),
                               e[4].elapsed_time(e[5]), e[5].elapsed_time(e[6])] for e in ev])
 
-    # ---- end-to-end through the Python API with host buffers: pinned h2d of the
-    # step's inputs into the captured step's buffers, the replay, and the d2h of
-    # its output, all inside the timed region
+    # ---- end-to-end through the Python API with host buffers, as a serving loop
+    # runs it: two buffer sets, each with its step captured (DecodeLayer.capture);
+    # step k copies its inputs from pinned host memory into set k % 2 on a copy
+    # stream, replays set k % 2's step, and copies its output back to pinned host
+    # memory on a third stream, so the copies of steps k + 1 and k - 1 overlap the
+    # compute of step k.  Every step's copies are inside the timed region.
+    graph2, inputs2, output2, device_error2 = second_set()
+    sets = [(graph, inputs, output), (graph2, inputs2, output2)]
     host_in = [t.cpu().pin_memory() for t in inputs]
-    out_host = torch.empty(output.shape, dtype=output.dtype).pin_memory()
+    out_host = [torch.empty(output.shape, dtype=output.dtype).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for i in range(2):
+        ev_done[i].record(stream)
+        ev_out[i].record(stream)
 
-    def e2e_step():
-        for d, hbuf in zip(inputs, host_in):
-            d.copy_(hbuf, non_blocking=True)
-        graph.replay()
-        out_host.copy_(output, non_blocking=True)
+    def e2e_step(k):
+        g, ins, out = sets[k % 2]
+        i = k % 2
+        s_in.wait_event(ev_done[i])          # step k - 2 has read this set's inputs
+        with torch.cuda.stream(s_in):
+            for d, hbuf in zip(ins, host_in):
+                d.copy_(hbuf, non_blocking=True)
+        ev_in[i].record(s_in)
+        stream.wait_event(ev_in[i])
+        stream.wait_event(ev_out[i])         # step k - 2's output has been copied out
+        g.replay()
+        ev_done[i].record(stream)
+        s_out.wait_event(ev_done[i])
+        with torch.cuda.stream(s_out):
+            out_host[i].copy_(out, non_blocking=True)
+        ev_out[i].record(s_out)
 
-    for _ in range(3):
-        e2e_step()
+    for k in range(4):
+        e2e_step(k)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(args.steps):
+        e2e_step(k)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     if clocks:
         clocks.stop()
-    st = device_error()
-    if st != 0:
-        raise RuntimeError(f"device error {L.STATUS.get(st)} in the end-to-end pass")
+    for err in (device_error(), device_error2()):
+        if err != 0:
+            raise RuntimeError(f"device error {L.STATUS.get(err)} in the end-to-end pass")
 
     elapsed, e2e_ms, attn_ms_total = max_over_ranks([elapsed, e2e_ms, per_call[:, 2].sum()],
                                                     world, dev)
@@ -526,8 +571,10 @@ def run_mine(args):
         "e2e": {"value": alg["rows"] * wl.n_heads * world / (e2e_ms / args.steps / 1e3),
                 "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": e2e_ms / args.steps,
-                "how": "per step: pinned host copies of the inputs into the step's buffers, "
-                       "StepGraph.replay(), pinned copy of the output back, one stream"},
+                "how": "per step: pinned host copies of the inputs into one of two buffer "
+                       "sets (copy stream), StepGraph.replay() of that set's captured step, "
+                       "pinned copy of the output back (third stream); copies of neighbouring "
+                       "steps overlap the compute"},
         "gpu_launches": launches * args.steps,
     }
     if rank == 0:
@@ -535,7 +582,7 @@ def run_mine(args):
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline_sample(wl, W, pc, h, q, lens)
         print(json.dumps(res), flush=True)
-    del graph
+    del graph, graph2, sets
     if world > 1:
         torch.distributed.destroy_process_group()
 
