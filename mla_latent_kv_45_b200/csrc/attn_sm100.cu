@@ -57,12 +57,6 @@ namespace {
 
 using namespace ptx;
 
-#ifndef MLA_ATTN_PREFETCH
-#define MLA_ATTN_PREFETCH 0   // steps of L2 prefetch ahead of the row ring (0 = none)
-#endif
-#ifndef MLA_ATTN_PV_FIRST
-#define MLA_ATTN_PV_FIRST 0   // 1: score MMAs of step i + 2 wait until P.V(i) is issued
-#endif
 
 constexpr int kHeads = 128;
 constexpr int kRow = 576;        // cached values per row
@@ -132,7 +126,6 @@ struct Bars {
   uint64_t drain_s, drain_pv;
   uint32_t tmem_base;
   volatile int abort;
-  volatile int pv_issued;     // even CTA: steps whose P.V MMAs have been issued
 };
 
 struct Ctx {
@@ -156,24 +149,6 @@ __device__ __forceinline__ bool wait_bar(const Ctx &c, uint64_t *bar, uint32_t p
     }
   }
 }
-
-#if MLA_ATTN_PV_FIRST
-// Bounded wait until a counter in this CTA's shared memory reaches `target`.
-__device__ __forceinline__ bool wait_count(const Ctx &c, volatile int *counter, int target) {
-  if (*counter >= target) return true;
-  const uint64_t t0 = globaltimer();
-  while (*counter < target) {
-    if (c.bars->abort) return false;
-    if (globaltimer() - t0 > kTimeoutNs) {
-      set_error(c.err, kErrTimeout);
-      c.bars->abort = 1;
-      return false;
-    }
-    __nanosleep(64);
-  }
-  return true;
-}
-#endif
 
 // Waits (bounded, ignoring the abort flag) for asynchronous work this CTA issued.
 __device__ __forceinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
@@ -323,9 +298,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_i8k,
                       const __grid_constant__ CUtensorMap tm_i8v, const AttnArgs a,
                       const float scale_log2) {
-#if MLA_ATTN_PREFETCH > 0
-  constexpr long kRowBytes = kI8 ? kI8Row : kRow * 2;
-#endif
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -362,7 +334,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(&bars->drain_s, 1);
     mbar_init(&bars->drain_pv, 1);
     bars->abort = 0;
-    bars->pv_issued = 0;
     fence_mbar_init();
   }
   if (warp == kWarpLoad && lane == 0) {
@@ -499,38 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int nk = 0;
       bool ok = true;
-#if MLA_ATTN_PREFETCH > 0
-      // this CTA's pages MLA_ATTN_PREFETCH steps ahead are brought into L2, so the
-      // row loads of the ring hit L2 instead of waiting a full DRAM latency
-      StepCursor ahead = cur;
-      for (int d = 0; d < MLA_ATTN_PREFETCH && ahead.valid; ++d) {
-        for (int sp = 0; sp < 2; ++sp) {
-          const int j = 2 * (int)rank + sp;
-          if (j < ahead.npages()) {
-            const int page = ahead.page(a, j);
-            if (page >= 0 && page < a.num_pages)
-              prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRowBytes,
-                          kPage * kRowBytes);
-          }
-        }
-        ahead.advance(a);
-      }
-#endif
       for (; cur.valid && ok; cur.advance(a)) {
-#if MLA_ATTN_PREFETCH > 0
-        if (ahead.valid) {
-          for (int sp = 0; sp < 2; ++sp) {
-            const int j = 2 * (int)rank + sp;
-            if (j < ahead.npages()) {
-              const int page = ahead.page(a, j);
-              if (page >= 0 && page < a.num_pages)
-                prefetch_l2(static_cast<const uint8_t *>(a.pool) + (size_t)page * kPage * kRowBytes,
-                            kPage * kRowBytes);
-            }
-          }
-          ahead.advance(a);
-        }
-#endif
         const int np = cur.npages();
         int pages[2];
         for (int sp = 0; sp < 2; ++sp) {
@@ -677,10 +617,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int sb = step & 1;
         // score buffer sb was last read by the softmax of step - 2
         if (step >= 2 && !wait_bar(ctx, &bars->s_free[sb], ((step >> 1) - 1) & 1)) break;
-#if MLA_ATTN_PV_FIRST
-        // keep P.V(step - 2) ahead of these score MMAs on the tensor pipe
-        if (step >= 2 && !wait_count(ctx, &bars->pv_issued, step - 1)) break;
-#endif
         const uint32_t sd = tmem + kTmemS + 128 * sb;
         for (int c = 0; c < 9; ++c, ++nk) {
           const int slot = nk % kKSlots;
@@ -741,9 +677,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         umma_commit_pair(&bars->pv_done, kBoth);
-#if MLA_ATTN_PV_FIRST
-        bars->pv_issued = step + 1;
-#endif
       }
       umma_commit_pair(&bars->drain_pv, 1);
       drain_bar(&bars->drain_pv, 0);

@@ -213,6 +213,38 @@ __global__ void __launch_bounds__(kThreads, 2)
       umma_commit(&bars->drain);
       gwait(bars, g.err, &bars->drain, 0);
     }
+  } else if (g.cluster) {
+    // epilogue of a split: this CTA's partial tile goes straight from TMEM into
+    // the shared memory of the CTA that owns its rows (see the reduction below)
+    const int quad = warp & 3;
+    const int ml = quad * 32 + lane;
+    const bool got = __all_sync(0xffffffffu, gwait(bars, g.err, &bars->acc_full[0], 0));
+    tc_fence_after();
+    cluster_arrive();   // this CTA's MMAs are complete: its stage ring may be overwritten
+    const int S = g.cluster, r = (int)cluster_ctarank();
+    const int rs = g.n_pad + 4;                      // row stride of a slice, floats
+    const int slice = 4 * ((32 + S - 1) / S) * rs;   // floats of one sender's slice
+    const int q = ml >> 2;                           // row quad of this thread's row
+    const int o = ((q + 1) * S - 1) / 32;            // owner: q_lo(o) <= q < q_hi(o)
+    const int rl = ml - 4 * (32 * o / S);
+    const uint32_t dst =
+        mapa(smem_u32(smem) + 4u * (uint32_t)(r * slice + rl * rs), (uint32_t)o);
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    cluster_wait();     // every CTA of the cluster is past its MMAs
+    if (got) {
+      for (int c = 0; c < g.n_pad; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          if (c + j < g.n_pad)   // the accumulator stride rounds n_pad up to 32
+            st_cluster_v4(dst + 4u * (uint32_t)(c + j), __uint_as_float(v[j]),
+                          __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                          __uint_as_float(v[j + 3]));
+      }
+    }
+    tc_fence_before();
   } else {
     // epilogue: warps 2..5 cover TMEM lanes 64..127, 0..63 (lane quadrant = warp % 4)
     const int quad = warp & 3;
@@ -229,15 +261,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint32_t r[32];
         tmem_ld32(taddr + c, r);
         tmem_wait_ld();
-        if (g.cluster) {
-          // this split's partial tile, [n][128 rows] fp32 at the start of the
-          // (drained) stage ring, for the in-cluster reduction below
-          float *tile = reinterpret_cast<float *>(smem);
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c + j < g.n_pad) tile[(c + j) * 128 + ml] = __uint_as_float(r[j]);
-          continue;
-        }
         if (m < P.M) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -258,29 +281,38 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive(&bars->acc_free[buf]);
     }
   }
-  __syncthreads();
   if (g.cluster) {
-    // In-cluster split-K reduction: CTA r of the S CTAs of this tile sums rows
-    // [4 q_lo, 4 q_hi) of all S partial tiles (split order 0..S-1, so the sum
-    // is deterministic) and writes the output.
-    cluster_sync();   // every partial tile written
+    // In-cluster split-K reduction.  The rows of the tile are cut into 32 quads
+    // of 4; CTA r of the S CTAs of this tile owns quads [q_lo, q_hi) =
+    // [32 r / S, 32 (r + 1) / S) and receives, in its drained stage ring, one
+    // slice [split][row][n] per split (written by that split's epilogue above).
+    // The owner sums the slices in split order 0..S-1 (deterministic) and
+    // writes the output.
+    if (warp < 2) {
+      __syncwarp();
+      cluster_arrive();
+      cluster_wait();
+    }
+    cluster_arrive();   // release: this CTA's slices are written
+    cluster_wait();     // acquire: all slices of this CTA's rows have landed
     const Item it = decode_item(g, item0);
     const GemmProblem &P = g.p[it.pi];
     const int S = g.cluster, r = (int)cluster_ctarank();
     const int q_lo = 32 * r / S, q_hi = 32 * (r + 1) / S, nq = q_hi - q_lo;
-    const uint32_t tile = smem_u32(smem);
+    const int rs = g.n_pad + 4, slice = 4 * ((32 + S - 1) / S) * rs;
+    const float *recv = reinterpret_cast<const float *>(smem);
     for (int u = threadIdx.x; u < g.n * nq; u += kThreads) {
-      const int n = u / nq, q = q_lo + u % nq;
-      const int m = it.m0 + 4 * q;
+      const int qq = u / g.n, n = u % g.n;
+      const int m = it.m0 + 4 * (q_lo + qq);
       if (m >= P.M) continue;
-      const uint32_t off = tile + (uint32_t)((n * 128 + 4 * q) * 4);
-      float4 acc = ld_cluster_v4(mapa(off, 0));
+      const float *p = recv + 4 * qq * rs + n;
+      float4 acc = make_float4(p[0], p[rs], p[2 * rs], p[3 * rs]);
       for (int sp = 1; sp < S; ++sp) {
-        const float4 v = ld_cluster_v4(mapa(off, (uint32_t)sp));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+        p += slice;
+        acc.x += p[0];
+        acc.y += p[rs];
+        acc.z += p[2 * rs];
+        acc.w += p[3 * rs];
       }
       const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
       if (P.out_mode == kOutBf16) {
@@ -294,8 +326,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         *reinterpret_cast<float4 *>(static_cast<float *>(P.out) + idx) = acc;
       }
     }
-    cluster_sync();   // no CTA leaves while another still reads its tile
   }
+  __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, g.tmem_cols);
@@ -364,8 +396,13 @@ namespace {
 cudaError_t set_smem_attr() {
   static api::PerDeviceOnce smem_attr;
   return smem_attr.run([] {
-    return cudaFuncSetAttribute(gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                232448);
+    const cudaError_t e = cudaFuncSetAttribute(
+        gemm_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1 / shared array as shared memory: two CTAs per SM
+    return cudaFuncSetAttribute(gemm_sm100_kernel,
+                                cudaFuncAttributePreferredSharedMemoryCarveout,
+                                cudaSharedmemCarveoutMaxShared);
   });
 }
 
@@ -433,7 +470,11 @@ int gemm_cluster_splits(int m_tiles, int heads, int k_chunks, int n) {
   const int tiles = m_tiles * heads;
   const int nn = n < 128 ? n : 128;   // cluster launches take the batch in chunks of 128
   const int n_pad = (nn + 15) / 16 * 16;
-  while (s > 2 && max_active_clusters(s, n_pad) < tiles) --s;
+  // The occupancy query counts one CTA of this kernel per SM (148 clusters of
+  // one on B200), while its launch bounds and shared memory place two; measured
+  // with 40 tiles, clusters of 6 (240 CTAs) ran in one wave and clusters of 7
+  // (280 CTAs, 30 clusters by twice the query's count) did not.
+  while (s > 2 && (2 * max_active_clusters(s, n_pad) < tiles || s * tiles > 2 * sm_count())) --s;
   const int per = (k_chunks + s - 1) / s;
   return (k_chunks + per - 1) / per;
 }
@@ -498,9 +539,13 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     const size_t smem = smem_for(g.n_pad);
     cudaError_t e;
     if (cluster) {
-      // one item per CTA; the splits of a tile form one cluster and their
-      // partial tiles ([n_pad][128] fp32) reuse the drained stage ring
-      if ((size_t)g.stages * stage_bytes < (size_t)g.n_pad * 128 * 4) return cudaErrorInvalidValue;
+      // one item per CTA; the splits of a tile form one cluster, and the slices
+      // they send each other ([split][rows][n_pad + 4] fp32) reuse the drained
+      // stage ring
+      const int S = ops[0].splits;
+      if ((size_t)g.stages * stage_bytes <
+          (size_t)S * 4 * ((32 + S - 1) / S) * (g.n_pad + 4) * 4)
+        return cudaErrorInvalidValue;
       g.cluster = ops[0].splits;
       g.items_per_cta = 1;
       e = launch_pdl_cluster(gemm_sm100_kernel, dim3(items), dim3(kThreads), smem, s, g.cluster,

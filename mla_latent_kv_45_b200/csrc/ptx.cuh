@@ -31,6 +31,17 @@ __device__ __forceinline__ void cluster_sync() {
                ::: "memory");
 }
 
+// The two halves of cluster_sync, for work placed between them: arrive
+// (release: this thread's earlier writes, shared::cluster ones included, are
+// visible to every thread that has waited) and wait (acquire).  Every thread of
+// every CTA of the cluster takes them in the same arrive / wait order.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
   uint32_t r;
@@ -128,12 +139,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-
-// Brings `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2
-// without touching shared memory.
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
@@ -317,6 +322,14 @@ __device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
                : "r"(addr)
                : "memory");
   return v;
+}
+
+// Four floats into shared memory of a CTA of the cluster (cluster address,
+// 16-byte aligned); ordered for the reader by a cluster barrier.
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
+               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 // Two floats into another CTA's shared memory, counted (8 bytes) on the
