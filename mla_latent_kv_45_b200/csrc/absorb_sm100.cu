@@ -46,6 +46,7 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: every bounded wait
 constexpr int kTile = 128 * 128;       // 128 rows x 64 bf16 (one A operand chunk)
 constexpr int kMaxStages = 6;
 constexpr int kSmemLimit = 232448;
+constexpr int kRopeAhead = 16;         // q_R pairs per epilogue thread with angles ahead (batch <= 64)
 
 struct Bars {
   uint64_t full[kMaxStages], empty[kMaxStages], acc1_full, qc_ready, acc2_full, drain;
@@ -118,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars->tmem_base, g.tmem_cols);
     tc_fence_before();
   }
+  __syncwarp();   // thread 0 alone set up the barriers
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
@@ -224,6 +226,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     grid_dep_wait();                       // positions and q_lat follow the predecessor
+    // The rotation angles of this thread's q_R pairs (w = tid + 128 k: sequence
+    // w / 32, pair w % 32) depend only on the positions: their cosines and sines
+    // are computed here, while the weights stream, instead of after the K loop.
+    const int half = g.rp.d_rope / 2;
+    const int tid = threadIdx.x - 64;
+    float rc[kRopeAhead], rsn[kRopeAhead];
+#pragma unroll
+    for (int k = 0; k < kRopeAhead; ++k) {
+      const int w = tid + 128 * k;
+      rc[k] = 1.f;
+      rsn[k] = 0.f;
+      if (w < g.n * half) rope_cos_sin(g.positions[g.n0 + w / half], g.rp.theta[w % half], rc[k], rsn[k]);
+    }
     uint8_t *qc = smem + g.off_qc;
     float *qr = reinterpret_cast<float *>(smem + g.off_qr);   // [n_pad][64]
     bool ok = await(bars, g.err, &bars->acc1_full, 0, g.timeout_ns);
@@ -261,17 +276,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     if (lane == 0 && !(g.skip_qc_arrive && quad == 0)) mbar_arrive(&bars->qc_ready);
     epi_sync();                            // q_R staging complete
-    // q_R,i rotated by the sequence's position, rounded once into q_lat
-    const int half = g.rp.d_rope / 2;
-    for (int w = threadIdx.x - 64; w < g.n * half; w += 128) {
+    // q_R,i rotated by the sequence's position in place in the staging tile,
+    // then rounded once into q_lat (each sequence's 64 values are one 128-byte
+    // line of q_lat: 16 threads store it, 8 bytes each)
+    auto rotate = [&](int w, float cf, float sf) {
       const int n = w / half, t = w % half;
       int j0, j1;
       rope_idx(g.rp, t, j0, j1);
       float x0 = qr[n * 64 + j0], x1 = qr[n * 64 + j1];
-      rope_pair(g.rp, t, g.positions[g.n0 + n], x0, x1);
-      __nv_bfloat16 *dst = g.q_lat + ((long)(g.n0 + n) * kH + head) * kRowLat + 512;
-      dst[j0] = __float2bfloat16_rn(x0);
-      dst[j1] = __float2bfloat16_rn(x1);
+      rope_rotate(cf, sf, x0, x1);
+      qr[n * 64 + j0] = x0;
+      qr[n * 64 + j1] = x1;
+    };
+#pragma unroll
+    for (int k = 0; k < kRopeAhead; ++k)
+      if (tid + 128 * k < g.n * half) rotate(tid + 128 * k, rc[k], rsn[k]);
+    for (int w = tid + 128 * kRopeAhead; w < g.n * half; w += 128) {
+      float cf, sf;
+      rope_cos_sin(g.positions[g.n0 + w / half], g.rp.theta[w % half], cf, sf);
+      rotate(w, cf, sf);
+    }
+    epi_sync();
+    for (int u = tid; u < g.n * 16; u += 128) {
+      const int n = u >> 4, j = (u & 15) * 4;
+      const float4 v = *reinterpret_cast<const float4 *>(qr + n * 64 + j);
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+      *reinterpret_cast<uint2 *>(g.q_lat + ((long)(g.n0 + n) * kH + head) * kRowLat + 512 + j) = pk;
     }
     ok = ok && await(bars, g.err, &bars->acc2_full, 0, g.timeout_ns);
     tc_fence_after();
@@ -291,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
   }
+  // the warps whose lane 0 alone ran a loop meet again before the CTA barrier
+  // (__syncthreads is warp-aligned: a warp must reach it converged)
+  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

@@ -348,6 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tmem_alloc_pair(&bars->tmem_base, kTmemCols);
     tc_fence_before();
   }
+  __syncwarp();   // thread 0 alone set up the barriers
   __syncthreads();
   tc_fence_after();
   cluster_sync();  // both CTAs' barriers exist before any remote access
@@ -889,6 +890,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   }
 
+  // the warps whose lane 0 alone ran a loop meet again before the CTA barrier
+  // (__syncthreads is warp-aligned: a warp must reach it converged)
+  __syncwarp();
   __syncthreads();
   cluster_sync();  // neither CTA touches the other's shared memory or TMEM any more
   if (warp == kWarpS) {

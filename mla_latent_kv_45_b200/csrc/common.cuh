@@ -31,19 +31,26 @@ template <> __device__ __forceinline__ __nv_bfloat16 st_cast<__nv_bfloat16>(floa
 
 __device__ __forceinline__ void set_error(int *err, int bit) { atomicOr(err, bit); }
 
-// cos / sin of the angle pos * theta in fp64.  The angle is first brought into
-// [-pi, pi] by Cody-Waite reduction with 2 pi split into a double and its
-// rounding remainder (exact enough for any int32 position), so the library
-// sincos only ever sees a small argument.
+// cos / sin of the angle pos * theta.  The angle is formed in fp64 and brought
+// into [-pi, pi] by Cody-Waite reduction with 2 pi split into a double and its
+// rounding remainder (exact enough for any int32 position); the reduced angle
+// is then rounded to fp32 (absolute error <= 2^-24 pi) and the fp32 library
+// sincosf takes it from there, so cf and sf are within a few 1e-7 of the exact
+// values, far below the bf16 rounding of every value they rotate.  (An fp64
+// sincos here is a long dependent chain of fp64 arithmetic on each thread.)
 __device__ __forceinline__ void rope_cos_sin(int pos, double theta, float &cf, float &sf) {
   const double a = (double)pos * theta;
   const double k = rint(a * 0.15915494309189535);      // a / (2 pi), rounded
   double r = fma(-k, 6.283185307179586, a);             // 2 pi, leading double
   r = fma(-k, 2.4492935982947064e-16, r);               // 2 pi minus its leading double
-  double s, c;
-  sincos(r, &s, &c);
-  cf = (float)c;
-  sf = (float)s;
+  sincosf((float)r, &sf, &cf);
+}
+
+// Rotates the pair (x0, x1) by the angle whose cosine and sine are (cf, sf).
+__device__ __forceinline__ void rope_rotate(float cf, float sf, float &x0, float &x1) {
+  const float a = x0, b = x1;
+  x0 = a * cf - b * sf;
+  x1 = a * sf + b * cf;
 }
 
 // Rotates the pair (x0, x1) by pos * theta_i.
@@ -51,9 +58,7 @@ __device__ __forceinline__ void rope_pair(const RopeParams &rp, int i, int pos, 
                                           float &x1) {
   float cf, sf;
   rope_cos_sin(pos, rp.theta[i], cf, sf);
-  const float a = x0, b = x1;
-  x0 = a * cf - b * sf;
-  x1 = a * sf + b * cf;
+  rope_rotate(cf, sf, x0, x1);
 }
 
 // Programmatic dependent launch.  A kernel launched with launch_pdl may start
@@ -131,10 +136,11 @@ __device__ __forceinline__ float warp_max(float v) {
 // Written by the plan kernel into the workspace, read by the attention and
 // combine kernels.
 struct PlanHeader {
-  int total_pages;   // sum over sequences of ceil(len / page_size)
-  int quota;         // pages per partition (last one may hold fewer)
+  int total_pages;   // sum over sequences of ceil(len / page_size) + gap (virtual pages)
+  int quota;         // virtual pages per partition (last one may hold fewer)
   int parts;         // partitions with work
   int num_partials;  // partial slots used by split sequences
+  int gap;           // virtual pages that stand for the fixed cost of each sequence
 };
 
 }  // namespace mla

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_alloc(&bars->tmem_base, g.tmem_cols);
     tc_fence_before();
   }
+  __syncwarp();   // thread 0 alone set up the barriers
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
@@ -222,26 +223,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     cluster_arrive();   // this CTA's MMAs are complete: its stage ring may be overwritten
     const int S = g.cluster, r = (int)cluster_ctarank();
-    const int rs = g.n_pad + 4;                      // row stride of a slice, floats
-    const int slice = 4 * ((32 + S - 1) / S) * rs;   // floats of one sender's slice
+    const int rp = 4 * ((32 + S - 1) / S);           // rows of an owner's share (padded)
+    const int slice = g.n_pad * rp;                  // floats of one sender's slice
     const int q = ml >> 2;                           // row quad of this thread's row
     const int o = ((q + 1) * S - 1) / 32;            // owner: q_lo(o) <= q < q_hi(o)
     const int rl = ml - 4 * (32 * o / S);
-    const uint32_t dst =
-        mapa(smem_u32(smem) + 4u * (uint32_t)(r * slice + rl * rs), (uint32_t)o);
+    const uint32_t dst = mapa(smem_u32(smem) + 4u * (uint32_t)(r * slice + rl), (uint32_t)o);
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     cluster_wait();     // every CTA of the cluster is past its MMAs
     if (got) {
+      // one float per column: the lanes of a warp (consecutive rows) write
+      // consecutive words of the owner's slice
       for (int c = 0; c < g.n_pad; c += 32) {
         uint32_t v[32];
         tmem_ld32(taddr + c, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
+        for (int j = 0; j < 32; ++j)
           if (c + j < g.n_pad)   // the accumulator stride rounds n_pad up to 32
-            st_cluster_v4(dst + 4u * (uint32_t)(c + j), __uint_as_float(v[j]),
-                          __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                          __uint_as_float(v[j + 3]));
+            st_cluster_f32(dst + 4u * (uint32_t)((c + j) * rp), __uint_as_float(v[j]));
       }
     }
     tc_fence_before();
@@ -285,9 +285,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     // In-cluster split-K reduction.  The rows of the tile are cut into 32 quads
     // of 4; CTA r of the S CTAs of this tile owns quads [q_lo, q_hi) =
     // [32 r / S, 32 (r + 1) / S) and receives, in its drained stage ring, one
-    // slice [split][row][n] per split (written by that split's epilogue above).
-    // The owner sums the slices in split order 0..S-1 (deterministic) and
-    // writes the output.
+    // slice [n][row] per split (written by that split's epilogue above).  The
+    // owner sums the slices in split order 0..S-1 (deterministic), four rows
+    // at a time, and writes the output.
     if (warp < 2) {
       __syncwarp();
       cluster_arrive();
@@ -299,20 +299,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     const GemmProblem &P = g.p[it.pi];
     const int S = g.cluster, r = (int)cluster_ctarank();
     const int q_lo = 32 * r / S, q_hi = 32 * (r + 1) / S, nq = q_hi - q_lo;
-    const int rs = g.n_pad + 4, slice = 4 * ((32 + S - 1) / S) * rs;
+    const int rp = 4 * ((32 + S - 1) / S), slice = g.n_pad * rp;
     const float *recv = reinterpret_cast<const float *>(smem);
     for (int u = threadIdx.x; u < g.n * nq; u += kThreads) {
-      const int qq = u / g.n, n = u % g.n;
+      const int qq = u % nq, n = u / nq;
       const int m = it.m0 + 4 * (q_lo + qq);
       if (m >= P.M) continue;
-      const float *p = recv + 4 * qq * rs + n;
-      float4 acc = make_float4(p[0], p[rs], p[2 * rs], p[3 * rs]);
+      const float *p = recv + n * rp + 4 * qq;
+      float4 acc = *reinterpret_cast<const float4 *>(p);
       for (int sp = 1; sp < S; ++sp) {
         p += slice;
-        acc.x += p[0];
-        acc.y += p[rs];
-        acc.z += p[2 * rs];
-        acc.w += p[3 * rs];
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
       const long idx = (long)n * P.ldy + (long)it.head * P.y_head + m;
       if (P.out_mode == kOutBf16) {
@@ -327,6 +328,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
+  // the warps whose lane 0 alone ran a loop meet again before the CTA barrier
+  // (__syncthreads is warp-aligned: a warp must reach it converged)
+  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -540,11 +544,10 @@ cudaError_t gemm(const GemmOp *ops, int nops, const __nv_bfloat16 *X, int n, lon
     cudaError_t e;
     if (cluster) {
       // one item per CTA; the splits of a tile form one cluster, and the slices
-      // they send each other ([split][rows][n_pad + 4] fp32) reuse the drained
-      // stage ring
+      // they send each other ([split][n_pad][rows] fp32) reuse the drained stage
+      // ring
       const int S = ops[0].splits;
-      if ((size_t)g.stages * stage_bytes <
-          (size_t)S * 4 * ((32 + S - 1) / S) * (g.n_pad + 4) * 4)
+      if ((size_t)g.stages * stage_bytes < (size_t)S * 4 * ((32 + S - 1) / S) * g.n_pad * 4)
         return cudaErrorInvalidValue;
       g.cluster = ops[0].splits;
       g.items_per_cta = 1;

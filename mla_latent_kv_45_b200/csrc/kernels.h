@@ -48,6 +48,7 @@ struct PlanArgs {
   int batch, page_size, max_pages;
   int parts_max, min_pages;
   int allow_empty;  // seq_len == 0 is an empty share (no rows), not an error
+  int gap;          // virtual pages charged per sequence (its fixed cost), 0 = none
   PlanHeader *hdr;
   int *seq_start;  // [batch + 1]
   int *part_base;  // [batch]
@@ -100,22 +101,26 @@ cudaError_t launch_merge_partials(const float *O, const float *m, const float *l
 namespace mla {
 
 // One piece of a partition: local pages [lp0, lp1) of sequence b (s0 = the
-// sequence's first global page, len = its row count).
+// virtual index of the sequence's first page, len = its row count).
 struct Segment {
   int b, lp0, lp1, len, s0;
 };
 
-// Walks the segments of partition p of the plan (global pages
-// [p*quota, (p+1)*quota) of the batch's concatenated page list).
+// Walks the segments of partition p of the plan: virtual pages
+// [p*quota, (p+1)*quota) of the batch's concatenated page list, in which each
+// sequence's pages are preceded by `gap` virtual pages that hold no rows (they
+// stand for the fixed cost of a sequence, so partitions with more sequences
+// get fewer pages).  Sequence b's pages are [seq_start[b], seq_start[b+1] - gap).
 struct SegmentWalker {
-  int g0, g1, b;
+  int g0, g1, b, gap;
 
   __device__ __forceinline__ void init(const AttnArgs &a, const PlanHeader &h, int p) {
     g0 = p * h.quota;
     g1 = min(h.total_pages, g0 + h.quota);
+    gap = h.gap;
     b = 0;
     if (g0 >= g1) return;
-    int lo = 0, hi = a.batch;  // seq_start[lo] <= g0 < seq_start[hi]
+    int lo = 0, hi = a.batch;  // the last b with seq_start[b] <= g0 (or 0)
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (a.seq_start[mid] <= g0) lo = mid; else hi = mid;
@@ -124,12 +129,14 @@ struct SegmentWalker {
   }
 
   __device__ __forceinline__ bool next(const AttnArgs &a, Segment &s) {
-    while (g0 < g1) {
-      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
-      if (s1 <= g0) { ++b; continue; }
+    while (g0 < g1 && b < a.batch) {
+      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1] - gap;
+      const int lo = max(g0, s0);
+      if (lo >= g1) return false;        // the range ends before sequence b's pages
+      if (s1 <= lo) { ++b; continue; }   // sequence b ends before lo (or has no pages)
       s.b = b;
       s.s0 = s0;
-      s.lp0 = g0 - s0;
+      s.lp0 = lo - s0;
       s.lp1 = min(g1, s1) - s0;
       s.len = a.seq_lens[b];
       g0 = s0 + s.lp1;

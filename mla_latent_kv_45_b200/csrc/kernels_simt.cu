@@ -316,9 +316,12 @@ template cudaError_t launch_rope_q<float>(const float *, int, int, int, const Ro
 // ---------------------------------------------------------------------------
 //
 // Sequence b holds n_b = ceil(len_b / page_size) pages.  Concatenating all
-// sequences' pages gives N pages; partition p takes global pages
-// [p*quota, (p+1)*quota).  A sequence cut by a partition boundary is computed
-// in pieces whose unnormalised partials are merged by the combine kernel.
+// sequences' pages, each preceded by `gap` virtual pages that stand for the
+// fixed cost of a sequence (its query load and its output), gives V virtual
+// pages; partition p takes virtual pages [p*quota, (p+1)*quota), so every
+// partition gets about the same cost, not the same number of pages.  A
+// sequence cut by a partition boundary is computed in pieces whose
+// unnormalised partials are merged by the combine kernel.
 
 __global__ void plan_kernel(PlanArgs a) {
   __shared__ int warp_tot[32];
@@ -329,14 +332,15 @@ __global__ void plan_kernel(PlanArgs a) {
   const long cap = (long)a.max_pages * a.page_size;
   if (tid == 0) carry = 0;
   __syncthreads();
-  // pass 1: page counts, validity, exclusive prefix sum -> seq_start
+  // pass 1: page counts, validity, exclusive prefix sum -> seq_start (the
+  // virtual index of each sequence's first page, after its gap)
   for (int base = 0; base < a.batch; base += blockDim.x) {
     const int b = base + tid;
     int n = 0;
     if (b < a.batch) {
       const int len = a.seq_lens[b];
       const bool ok = len > 0 && len <= cap;
-      n = ok ? (len + a.page_size - 1) / a.page_size : 0;
+      n = (ok ? (len + a.page_size - 1) / a.page_size : 0) + a.gap;
       a.bad[b] = ok ? 0 : 1;
       // an empty share of a sequence split across devices is not an error
       if (!ok && !(a.allow_empty && len == 0)) set_error(a.err, kErrRange);
@@ -359,27 +363,29 @@ __global__ void plan_kernel(PlanArgs a) {
     }
     __syncthreads();
     const int incl = v + ((tid >> 5) ? warp_tot[(tid >> 5) - 1] : 0) + carry;
-    if (b < a.batch) a.seq_start[b] = incl - n;
+    if (b < a.batch) a.seq_start[b] = incl - n + a.gap;
     __syncthreads();
     if (tid == blockDim.x - 1) carry = incl;
     __syncthreads();
   }
   __shared__ int quota;
   if (tid == 0) {
-    const int N = carry;
-    a.seq_start[a.batch] = N;
+    const int V = carry;                     // virtual pages
+    const int N = V - a.batch * a.gap;       // cache pages
+    a.seq_start[a.batch] = V + a.gap;
     int parts = 0, q = 1;
     if (N > 0) {
       int p = a.parts_max;
       const int by_min = (N + a.min_pages - 1) / a.min_pages;
       if (p > by_min) p = by_min;
       if (p < 1) p = 1;
-      q = (N + p - 1) / p;
-      parts = (N + q - 1) / q;
+      q = (V + p - 1) / p;
+      parts = (V + q - 1) / q;
     }
-    a.hdr->total_pages = N;
+    a.hdr->total_pages = N > 0 ? V : 0;
     a.hdr->quota = q;
     a.hdr->parts = parts;
+    a.hdr->gap = a.gap;
     quota = q;
     carry = 0;
   }
@@ -389,7 +395,7 @@ __global__ void plan_kernel(PlanArgs a) {
     const int b = base + tid;
     int pieces = 0;
     if (b < a.batch) {
-      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+      const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1] - a.gap;
       if (s1 > s0) pieces = (s1 - 1) / quota - s0 / quota + 1;
     }
     const int n = pieces > 1 ? pieces : 0;
@@ -444,16 +450,19 @@ __global__ void attn_simt(AttnArgs a) {
   constexpr int MAXD = 8;  // d_c <= MAXD * NT
   const int g1 = min(hdr.total_pages, (p + 1) * hdr.quota);
   int g0 = p * hdr.quota;
-  // first sequence: largest b with seq_start[b] <= g0
-  int lo = 0, hi = a.batch;  // invariant seq_start[lo] <= g0 < seq_start[hi]
+  // first sequence: the last b with seq_start[b] <= g0 (or 0)
+  int lo = 0, hi = a.batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (a.seq_start[mid] <= g0) lo = mid; else hi = mid;
   }
   int b = lo;
-  while (g0 < g1) {
-    const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
-    if (s1 <= g0) { ++b; continue; }
+  while (g0 < g1 && b < a.batch) {
+    const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1] - hdr.gap;
+    const int first = max(g0, s0);
+    if (first >= g1) break;                 // the range ends before sequence b's pages
+    if (s1 <= first) { ++b; continue; }     // sequence b ends before (or has no pages)
+    g0 = first;
     const int lp1 = min(g1, s1) - s0;
     const int len = a.seq_lens[b];
     const int r_begin = (g0 - s0) * a.page_size;
@@ -617,7 +626,7 @@ __global__ void combine_kernel(AttnArgs a) {
   const int pb = a.part_base[b];
   if (pb < 0) return;
   const PlanHeader hdr = *a.hdr;
-  const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1];
+  const int s0 = a.seq_start[b], s1 = a.seq_start[b + 1] - hdr.gap;
   const int pieces = (s1 - 1) / hdr.quota - s0 / hdr.quota + 1;
   const float *pm = a.part_m + (long)pb * a.n_heads + h;   // piece j at pm[j * n_heads]
   const float *pl = a.part_l + (long)pb * a.n_heads + h;

@@ -124,6 +124,7 @@ mla_status decode_attn_impl(const mla_dims *dims, const mla_paged_cache *cache, 
   pa.max_pages = cache->max_pages_per_seq;
   pa.parts_max = parts;
   pa.min_pages = d.dtype == MLA_BF16 ? sm100::kAttnMinPages : 1;
+  pa.gap = d.dtype == MLA_BF16 ? sm100::kAttnSeqGap : 0;
   pa.allow_empty = pO != nullptr;
   pa.hdr = reinterpret_cast<PlanHeader *>(at(ws, L.hdr));
   pa.seq_start = reinterpret_cast<int *>(at(ws, L.seq_start));

@@ -121,6 +121,7 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_dims *dims, const mla_pa
   pa.max_pages = cache->max_pages_per_seq;
   pa.parts_max = parts;
   pa.min_pages = d.dtype == MLA_BF16 ? sm100::kAttnMinPages : 1;
+  pa.gap = d.dtype == MLA_BF16 ? sm100::kAttnSeqGap : 0;
   pa.hdr = reinterpret_cast<PlanHeader *>(ws + R.hdr);
   pa.seq_start = reinterpret_cast<int *>(ws + R.seq_start);
   pa.part_base = reinterpret_cast<int *>(ws + R.part_base);

@@ -324,12 +324,10 @@ __device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
   return v;
 }
 
-// Four floats into shared memory of a CTA of the cluster (cluster address,
-// 16-byte aligned); ordered for the reader by a cluster barrier.
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};"
-               ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+// A float into shared memory of a CTA of the cluster (cluster address);
+// ordered for the reader by a cluster barrier.
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(a) : "memory");
 }
 
 // Two floats into another CTA's shared memory, counted (8 bytes) on the

@@ -16,6 +16,13 @@ namespace sm100 {
 // less work than this is merged away by the plan).
 constexpr int kAttnMinPages = 4;
 
+// Virtual pages the plan charges each sequence for its fixed cost in the
+// attention kernel (loading its q_lat, draining the pipeline at its end and
+// writing its output).  Measured on B200 over the 74 partitions of a batch of
+// 64 sequences (1024..8192 rows): a partition takes about 4.4 us per step of 4
+// pages plus 5.5 us per sequence piece, so a piece costs about 5 pages.
+constexpr int kAttnSeqGap = 5;
+
 // [W_DKV h_b ; W_KR h_b] in fp32 into xkv [batch][576].
 cudaError_t append_proj(const __nv_bfloat16 *h, const __nv_bfloat16 *W_DKV,
                         const __nv_bfloat16 *W_KR, int batch, int d_model, float *xkv, int *err,
