@@ -153,6 +153,23 @@ def test_bf16_attn_step_tails(splits):
         np.testing.assert_allclose(lh[b], lr, atol=LSE_ATOL, rtol=LSE_RTOL)
 
 
+@pytest.mark.parametrize("splits", [0, 5, 40])
+def test_bf16_attn_cost_balanced_plan_edges(splits):
+    """The plan charges each sequence a few virtual pages with no rows, so a
+    partition's range may start or end inside those, hold no rows at all, or
+    cut a sequence anywhere: many one- and two-page sequences around a few long
+    ones, with few and with many partitions."""
+    lens = np.array([1, 64, 65, 2, 3000, 1, 1, 128, 129, 7, 1, 700, 64, 1, 2, 5000, 1, 63, 1, 2])
+    wl, pc, q, z, lse, st = attn_case(lens, splits)
+    assert st == 0
+    od = oracle_dims(wl)
+    zh, lh = host(z), host(lse)
+    for b, Lb in enumerate(lens):
+        zr, lr = oracle.attend_latent(q[b], pc.rows_f32(b, Lb), od)
+        assert_bf16_close(zh[b], zr, f"z seq {b} len {Lb}")
+        np.testing.assert_allclose(lh[b], lr, atol=LSE_ATOL, rtol=LSE_RTOL)
+
+
 def test_bf16_attn_split_and_page_order_invariance():
     lens = np.array([900, 5, 300, 2000])
     _, _, _, z1, l1, _ = attn_case(lens, 1)
