@@ -327,8 +327,13 @@ __global__ void plan_kernel(PlanArgs a) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
   const int tid = threadIdx.x;
-  grid_dep_launch();   // the attention kernel may launch and set up meanwhile
+  // The attention kernel may launch once this kernel's predecessor is done, not
+  // before: launched earlier, its CTAs (a whole SM's shared memory each) take SMs
+  // that the predecessor's own pending CTAs are waiting for.  Measured on the
+  // v2_batch64 step issued on one stream: 216 us with the early trigger, 203 us
+  // with this order.
   grid_dep_wait();
+  grid_dep_launch();
   const long cap = (long)a.max_pages * a.page_size;
   if (tid == 0) carry = 0;
   __syncthreads();
