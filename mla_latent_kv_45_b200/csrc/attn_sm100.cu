@@ -369,7 +369,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true, pend = false, pend_has[2] = {false, false};
     float pend_sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
     // chunk idx (in `slot`) landed: int8 codes of page sp at +8 KB + 4 KB sp, row r
-    // at 64 r; bf16 out at +8 KB sp, row r at 128 r, 16-byte unit u at (u ^ (r & 7)) << 4.
+    // at 64 r, its 16-byte unit u at (u ^ ((r >> 1) & 3)) << 4 (64-byte swizzle: the
+    // lanes of a warp, one row each, read distinct banks); bf16 out at +8 KB sp,
+    // row r at 128 r, 16-byte unit u at (u ^ (r & 7)) << 4.
     // Page 1's output covers page 0's input and, from row 32 on, its own: page 0
     // is converted first, and every 32-row batch is read before it is written.
     auto finish_k = [&](int slot, int idx, int c, const bool (&has)[2],
@@ -381,10 +383,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!has[sp]) continue;
           for (int hf = 0; hf < 2; ++hf) {
             const int r = 32 * hf + lane;
-            const uint4 *in = reinterpret_cast<const uint4 *>(base + 8192 + 4096 * sp + 64 * r);
+            const uint8_t *in = base + 8192 + 4096 * sp + 64 * r;
             uint4 v[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = in[j];
+            for (int j = 0; j < 4; ++j)
+              v[j] = *reinterpret_cast<const uint4 *>(in + ((j ^ ((r >> 1) & 3)) << 4));
             __syncwarp();
             uint8_t *out = base + kBox * sp + 128 * r;
 #pragma unroll
@@ -514,17 +517,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto finish = [&](int slot, int idx, int valid, float sc0, float sc1) -> bool {
       if (!wait_bar(ctx, &bars->v_land[slot], (idx / kVSlots) & 1)) return false;
       if (kI8) {
-        // int8 codes of row r at +8 KB + 128 r (128 latent columns) -> bf16 boxes
-        // 0 (columns 0-63) at 128 r and 1 (64-127) at 8 KB + 128 r: box 1's row r is
-        // exactly the input row r, which the lane has read before it writes
+        // int8 codes of row r at +8 KB + 128 r (128 latent columns, 16-byte unit j
+        // at (j ^ (r & 7)) << 4: 128-byte swizzle, so the lanes read distinct banks)
+        // -> bf16 boxes 0 (columns 0-63) at 128 r and 1 (64-127) at 8 KB + 128 r: box
+        // 1's row r is exactly the input row r, which the lane has read before it writes
         uint8_t *dst = smem + kOffV + slot * kVChunk;
         for (int hf = 0; hf < 2; ++hf) {
           const int r = 32 * hf + lane;
           const float sc = hf ? sc1 : sc0;
           uint4 v[8];
-          const uint4 *in = reinterpret_cast<const uint4 *>(dst + kBox + 128 * r);
+          const uint8_t *in = dst + kBox + 128 * r;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = in[j];
+          for (int j = 0; j < 8; ++j)
+            v[j] = *reinterpret_cast<const uint4 *>(in + ((j ^ (r & 7)) << 4));
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
@@ -966,8 +971,8 @@ cudaError_t launch_attn_t(const AttnArgs &a, int parts, cudaStream_t s) {
     // k_R (bytes 512..639) as swizzled bf16 boxes; the codes in plain boxes that
     // the kernel converts
     if (!make_map_i8(&tm_rows, a.pool, pool_rows, 128, kPage, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_i8(&tm_i8k, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_i8(&tm_i8v, a.pool, pool_rows, 128, kPage, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !make_map_i8(&tm_i8k, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_i8(&tm_i8v, a.pool, pool_rows, 128, kPage, CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   } else {
     if (!make_map(&tm_rows, a.pool, pool_rows, 64, kPage, CU_TENSOR_MAP_SWIZZLE_128B))
