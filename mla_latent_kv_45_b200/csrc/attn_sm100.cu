@@ -39,8 +39,9 @@
 //  * Warps 0-7 softmax + epilogue; warp 8 loads score rows; warp 9 TMEM
 //    allocation, q_lat loads and (even CTA) the score MMAs; warp 10 (even CTA)
 //    the P.V MMAs; warp 11 the latent-column loads for P.V.
-//  * Partitions come from the plan kernel (equal page counts); a sequence cut
-//    by a partition boundary writes an unnormalised partial that the combine
+//  * Partitions come from the plan kernel (equal cost: each sequence counts a
+//    few virtual pages for its fixed cost besides its pages); a sequence cut by
+//    a partition boundary writes an unnormalised partial that the combine
 //    kernel merges.
 //  * Every wait is bounded (globaltimer); on expiry the kernel records
 //    kErrTimeout in the error word, stops issuing work, drains what it issued
