@@ -102,6 +102,32 @@ def test_tiny_fp32_decode_loop_matches_naive_forward():
 # bf16, DeepSeek-V2 head / latent sizes
 # ---------------------------------------------------------------------------
 
+def test_bf16_decode_loop_matches_naive_forward():
+    """Multi-step decode at the DeepSeek-V2 sizes: 24 steps from an empty cache,
+    each appending its row through the library and attending over the rows the
+    library appended before, against the oracle's causal whole-sequence forward
+    (K and V rebuilt, fp64)."""
+    wl = synth.reduced(synth.V2_BATCH64, "v2_loop", 27, 2, 0, 0)
+    W = synth.make_weights(wl)
+    T = 24
+    hs = synth.make_hidden(wl, n=wl.batch * T).reshape(wl.batch, T, wl.d_model)
+    dims, od = lib_dims(wl), oracle_dims(wl)
+    pc = synth.make_paged_cache(dataclasses.replace(wl, new_tokens=T), np.zeros(wl.batch, dtype=np.int64),
+                                fill=False)
+    lens = torch.zeros(wl.batch, dtype=torch.int32, device="cuda")
+    cache = dev_cache(pc, np.zeros(wl.batch))
+    cache.seq_lens = lens
+    layer = DecodeLayer(dims, dev_weights(W, wl), wl.batch)
+    outs = []
+    for t in range(T):
+        lens.fill_(t + 1)
+        outs.append(host(layer.step(cache, dev(hs[:, t], wl), ipos([t] * wl.batch))).copy())
+    assert layer.device_error() == 0
+    for b in range(wl.batch):
+        ref = oracle.forward_naive(hs[b], W, od)
+        assert_bf16_close(np.stack([o[b] for o in outs]), ref, f"seq {b}")
+
+
 V2R = synth.reduced(synth.V2_BATCH64, "v2_ragged", 20, 6, 0, 0)
 RAGGED = np.array([1, 63, 64, 65, 700, 129])
 
