@@ -93,6 +93,36 @@ def test_noalloc_matches_oracle_and_workspace_entry_point(kind, splits):
         np.testing.assert_allclose(lh, host(lse_ws), atol=LSE_ATOL, rtol=LSE_RTOL)
 
 
+def test_noalloc_int8_pool_matches_oracle_and_workspace_entry_point():
+    """The same entry point over an int8-row pool (MLA_CACHE_INT8)."""
+    lens = np.array([1, 700, 5000, 64, 129])
+    wl = synth.reduced(synth.V2_BATCH64, "noalloc_int8", 54, len(lens), 0, 0, new_tokens=0)
+    pc = synth.make_paged_cache_int8(wl, lens, spare_pages=1)
+    q_host = synth.make_q_lat(wl)
+    q = dev(q_host, wl)
+    dims = dataclasses.replace(lib_dims(wl), cache_format=L.MLA_CACHE_INT8)
+    cache = L.PagedCache(torch.from_numpy(pc.pool).cuda(),
+                         torch.from_numpy(np.ascontiguousarray(pc.block_table, dtype=np.int32)).cuda(),
+                         torch.from_numpy(lens.astype(np.int32)).cuda())
+    od = oracle_dims(wl)
+    ref = []
+    for b, Lb in enumerate(lens):
+        codes, exps, k_r = pc.fields(b, Lb)
+        rows = np.concatenate([oracle.dequantize_int8_pow2(codes, exps), k_r], axis=1)
+        ref.append(oracle.attend_latent(q_host[b], rows, od))
+    z_ws, lse_ws = _with_workspace(dims, cache, q, wl.batch)
+    z = torch.empty_like(z_ws)
+    lse = torch.empty_like(lse_ws)
+    assert _noalloc_c_abi(dims, cache, q, z, lse) == 0
+    assert _noalloc_status() == 0
+    zh, lh = host(z), host(lse)
+    for b in range(wl.batch):
+        assert_bf16_close(zh[b], ref[b][0], f"z seq {b}")
+        np.testing.assert_allclose(lh[b], ref[b][1], atol=LSE_ATOL, rtol=LSE_RTOL)
+    assert_bf16_close(zh, host(z_ws), "z vs workspace entry point")
+    np.testing.assert_allclose(lh, host(lse_ws), atol=LSE_ATOL, rtol=LSE_RTOL)
+
+
 def test_noalloc_reports_device_range_errors():
     lens = np.array([100, 130])
     wl = synth.reduced(synth.V2_BATCH64, "noalloc_bad", 53, 2, 0, 0, new_tokens=0)
