@@ -61,12 +61,38 @@ LAUNCHES_FULL_STEP = 9
 LAUNCHES_ATTENTION = 3
 
 
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _find_number(obj, key):
+    """The first number stored under ``key`` anywhere in a parsed JSON value."""
+    if isinstance(obj, dict):
+        v = obj.get(key)
+        if isinstance(v, (int, float)) and not isinstance(v, bool):
+            return float(v)
+        for x in obj.values():
+            r = _find_number(x, key)
+            if r is not None:
+                return r
+    elif isinstance(obj, list):
+        for x in obj:
+            r = _find_number(x, key)
+            if r is not None:
+                return r
+    return None
+
+
+def peaks(path=None):
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source): the measured
+    peaks of this machine's B200s when MEASURED_PEAKS.json holds them (at any depth),
+    else the pool's earlier measurement."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+            hbm, tf = _find_number(d, "hbm_gbs"), _find_number(d, "bf16_tflops")
+            if hbm and tf:
+                return hbm, tf, _find_number(d, "bf16_tflops_sustained"), "measured"
+        except (OSError, ValueError):
+            pass
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 

@@ -90,3 +90,24 @@ def test_prefill_chunk_reads_each_row_once():
     cached = wl.batch * (wl.prior_max + T)
     assert got["attn_bytes"] == cached * 1152 + wl.batch * T * H * (576 + 512) * 2
     assert got["attn_flops"] == int(lens.sum()) * H * 2176
+
+
+def test_measured_peaks_file_layouts(tmp_path):
+    """The roofline's denominators come from MEASURED_PEAKS.json when it holds
+    them, at any depth of the file; anything else falls back, never fails."""
+    import json
+    flat = tmp_path / "flat.json"
+    flat.write_text(json.dumps({"hbm_gbs": 6542.1, "bf16_tflops": 1641.8,
+                                "bf16_tflops_sustained": 1367.1}))
+    assert bench.peaks(str(flat)) == (6542.1, 1641.8, 1367.1, "measured")
+    nested = tmp_path / "nested.json"
+    nested.write_text(json.dumps({"gpu": "B200", "peaks": {"hbm_gbs": 6500, "bf16_tflops": 1600}}))
+    hbm, tf, sus, src = bench.peaks(str(nested))
+    assert (hbm, tf, sus, src) == (6500.0, 1600.0, None, "measured")
+    missing = tmp_path / "missing.json"
+    missing.write_text(json.dumps({"hbm_gbs": 6500}))
+    assert bench.peaks(str(missing))[3] == "fallback"
+    broken = tmp_path / "broken.json"
+    broken.write_text("{not json")
+    assert bench.peaks(str(broken))[3] == "fallback"
+    assert bench.peaks(str(tmp_path / "absent.json"))[3] == "fallback"
