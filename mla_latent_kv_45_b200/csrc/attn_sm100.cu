@@ -838,7 +838,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       ok = ok && wait_bar(ctx, &bars->lx, tc.nseg & 1);
       const float2 px = reinterpret_cast<const float2 *>(lx + 64 * g)[lane];
       const float f0 = s0 + px.x, f1 = s1 + px.y;   // same sum in both CTAs
-      if (quad == 0) reinterpret_cast<float2 *>(lsum + 64 * g)[lane] = make_float2(f0, f1);
+      // one division per head: z is O^T times the reciprocal of its row sum
+      // (a division per output value kept the softmax warps 4 us longer per call)
+      if (quad == 0) reinterpret_cast<float2 *>(lsum + 64 * g)[lane] = make_float2(1.f / f0, 1.f / f1);
       const int b = tc.seg.b;
       const int pbase = a.part_base[b];
       const bool whole = pbase < 0;
@@ -867,7 +869,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       }
       ok = ok && wait_bar(ctx, &bars->pv_done, i & 1);
-      softmax_sync();                        // lsum complete for both halves
+      softmax_sync();                        // 1 / l complete for both halves
       tc_fence_after();
       const int col = 256 * g + 128 * (int)rank + quad * 32 + lane;   // latent column of my lane
       const uint32_t ob = tmem + lane_off + kTmemO + 128 * g;
@@ -879,7 +881,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + (long)b * kHeads * kDc + col;
 #pragma unroll
           for (int kk = 0; kk < 32; ++kk)
-            z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] / lsum[c + kk]);
+            z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] * lsum[c + kk]);
         } else {
           float *o = pO + col;
 #pragma unroll
