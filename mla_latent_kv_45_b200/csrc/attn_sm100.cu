@@ -90,8 +90,8 @@ constexpr int kOffRed = kOffStg + kStgBytes;   // [2 halves][4 warps][64] floats
 constexpr int kOffX = kOffRed + 2048;          // [2 parities][128] the partner's tile maxima
 constexpr int kOffMb = kOffX + 1024;           // [8 warps][64] running max, per warp
 constexpr int kOffAlpha = kOffMb + 2048;       // [128] rescale factors
-constexpr int kOffLsum = kOffAlpha + 512;      // [128] row sums of the pair
-constexpr int kOffLx = kOffLsum + 512;         // [128] the partner's row sums
+constexpr int kOffLinv = kOffAlpha + 512;      // [128] 1 / row sum of the pair, per head
+constexpr int kOffLx = kOffLinv + 512;         // [128] the partner's row sums
 constexpr int kOffBar = kOffLx + 512;
 constexpr int kSmemBytes = kOffBar + 512 + 1024;
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0 &&
@@ -700,7 +700,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float *xmax = reinterpret_cast<float *>(smem + kOffX);
     float *mb = reinterpret_cast<float *>(smem + kOffMb) + warp * 64;
     float *alpha_s = reinterpret_cast<float *>(smem + kOffAlpha);
-    float *lsum = reinterpret_cast<float *>(smem + kOffLsum);
+    float *linv = reinterpret_cast<float *>(smem + kOffLinv);
     float *lx = reinterpret_cast<float *>(smem + kOffLx);
     const bool outgoing = g != (int)rank;    // this half of P is the partner's B operand
     float m0 = -INFINITY, m1 = -INFINITY;    // running max (log2 units) of heads 64g + 2 lane, +1
@@ -840,7 +840,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const float f0 = s0 + px.x, f1 = s1 + px.y;   // same sum in both CTAs
       // one division per head: z is O^T times the reciprocal of its row sum
       // (a division per output value kept the softmax warps 4 us longer per call)
-      if (quad == 0) reinterpret_cast<float2 *>(lsum + 64 * g)[lane] = make_float2(1.f / f0, 1.f / f1);
+      if (quad == 0) reinterpret_cast<float2 *>(linv + 64 * g)[lane] = make_float2(1.f / f0, 1.f / f1);
       const int b = tc.seg.b;
       const int pbase = a.part_base[b];
       const bool whole = pbase < 0;
@@ -881,7 +881,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           __nv_bfloat16 *z = reinterpret_cast<__nv_bfloat16 *>(a.z) + (long)b * kHeads * kDc + col;
 #pragma unroll
           for (int kk = 0; kk < 32; ++kk)
-            z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] * lsum[c + kk]);
+            z[(long)(c + kk) * kDc] = __float2bfloat16_rn(ov[kk] * linv[c + kk]);
         } else {
           float *o = pO + col;
 #pragma unroll
