@@ -314,16 +314,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 
 // ---------------------------------------------------------------- DSMEM
 
-// Four floats from shared memory of a CTA of the cluster (cluster address).
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
-}
-
 // A float into shared memory of a CTA of the cluster (cluster address);
 // ordered for the reader by a cluster barrier.
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float a) {
